@@ -1,0 +1,470 @@
+"""Benchmark of the Velox geometry-routed attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload headline|sweep] [--P 48]
+
+One step = one pass of the whole hot path over one chunk's synthetic inputs,
+with the KV cache resident in HBM: frustum slices of every past chunk, slice
+overlap counts, geometry-modulated top-k routing (pooling + scores + select)
+and block-sparse attention over the routed blocks. `value` is the whole-job
+throughput in TFLOP/s of attention work on the kept blocks
+(4 * B * H * m * topk * T^2 * d per step) divided by the step time. The dense
+attention over every block (the build's own dense baseline) is timed
+separately for the speedup.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own chunk
+(seed + rank) -- heads/chunks are independent units, there is no data-path
+collective -- and the time is the max over ranks ("scaling": "weak").
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the oracle stands in for a reference
+implementation: the method's pages publish no code).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from geometry_routed_block_b200 import synth  # noqa: E402
+
+METRIC = "chunk-48 routed attention ms & TFLOP/s (kept blocks), speedup vs dense; routing GB/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_desc(s: synth.Shape) -> str:
+    return (f"chunk-{s.P} routed attention: B{s.B} H{s.H} d{s.d} T{s.T}, chunk {s.F}x{s.Hp}x{s.Wp}"
+            f"={s.Nq} tokens, {s.P} past chunks, Nk={s.Nk}, {s.nKB} key blocks, topk={s.topk}, "
+            f"alpha={s.alpha}")
+
+
+def kept_flops(s: synth.Shape) -> float:
+    return 4.0 * s.B * s.H * s.m * s.topk * s.T * s.T * s.d
+
+
+def dense_flops(s: synth.Shape) -> float:
+    return 4.0 * s.B * s.H * s.m * s.nKB * s.T * s.T * s.d
+
+
+def routing_bytes(s: synth.Shape) -> float:
+    """Algorithmic bytes of routing: Q + past K read once, idx written, counts read."""
+    return (2.0 * s.B * s.H * s.d * (s.Nq + s.P * s.Nq) + 4.0 * s.B * s.H * s.m * s.topk
+            + 4.0 * s.B * s.m * s.P)
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle sample (cpu_baseline and the reference arm)
+# ----------------------------------------------------------------------------
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(case, head: int = 0, n_rows: int | None = None):
+    """Runs the oracle on: all geometry (slices + overlap counts), the routing
+    of one (batch, head) pair and the attention of `n_rows` query blocks of
+    that pair (all of them by default). Returns (estimated whole-step seconds,
+    sample seconds, description); the estimate scales the per-head routing by
+    B*H and the per-row attention by B*H*m."""
+    from oracle import velox_oracle as vo
+    s = case.shape
+    n_rows = s.m if n_rows is None else max(1, min(s.m, n_rows))
+    t0 = time.perf_counter()
+    sl = vo.slices_build(case.past_depth[0], case.past_poses[0], case.past_intr[0])
+    counts = vo.block_overlap(case.cur_depth, case.cur_cam, sl[None], s.F, s.T)
+    t1 = time.perf_counter()
+    q, k, v = case.q[0][:, head:head + 1], case.k[0][:, head:head + 1], case.v[0][:, head:head + 1]
+    idx, _ = vo.route_topk(q, k, counts, s.alpha, s.topk, s.T)
+    t2 = time.perf_counter()
+    step = max(1, s.m // n_rows)
+    rows = [(0, 0, qb) for qb in range(0, s.m, step)][:n_rows]
+    vo.sparse_attention(q, k, v, idx, s.T, rows=rows)
+    t3 = time.perf_counter()
+    pairs = s.B * s.H
+    est = (t1 - t0) + pairs * (t2 - t1) + pairs * s.m * (t3 - t2) / len(rows)
+    desc = (f"oracle (numpy fp64): all geometry, routing of 1 of {pairs} (batch, head) pairs and "
+            f"attention of {len(rows)} of its {s.m} query blocks; step time = geometry + "
+            f"{pairs} x routing + {pairs * s.m} x per-block attention")
+    return est, t3 - t0, desc
+
+
+# ----------------------------------------------------------------------------
+# GPU workload
+# ----------------------------------------------------------------------------
+
+class Workload:
+    def __init__(self, case, device):
+        import torch
+        from geometry_routed_block_b200 import velox as vx
+        self.vx, self.torch = vx, torch
+        self.case, self.s = case, case.shape
+        s = self.s
+        self.device = device
+
+        def dev(a):
+            if a.dtype == np.uint16:
+                return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(
+                    torch.bfloat16).to(device)
+            return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+        self.q, self.k, self.v = dev(case.q[0]), dev(case.k[0]), dev(case.v[0])
+        self.past_depth = dev(case.past_depth[0])
+        self.past_poses = dev(case.past_poses[0])
+        self.past_intr = dev(case.past_intr[0])
+        self.cur_depth, self.cur_cam = dev(case.cur_depth), dev(case.cur_cam)
+        self.slices = torch.empty((s.P, 18), dtype=torch.float32, device=device)
+        self.counts = torch.empty((s.B, s.m, s.P), dtype=torch.int32, device=device)
+        self.ws = vx.route_workspace(s.B, s.H, s.Nq, s.Nk, s.d, s.T, device)
+        self.idx = torch.empty((s.B, s.H, s.m, s.topk), dtype=torch.int32, device=device)
+        self.o = torch.empty_like(self.q)
+        self.o_dense = torch.empty_like(self.q)
+        self.lse = torch.empty((s.B, s.H, s.Nq), dtype=torch.float32, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.launches_per_step = 6  # slices, overlap, pool_q, pool_score, select, attention
+
+    def geometry(self):
+        vx, s = self.vx, self.s
+        vx.slices_build(self.past_depth, self.past_poses, self.past_intr, out=self.slices)
+        vx.block_overlap(self.cur_depth, self.cur_cam, self.slices[None], s.F, s.T, out=self.counts)
+
+    def route(self):
+        s = self.s
+        self.vx.route_topk(self.q, self.k, self.counts, s.alpha, s.topk, s.T, ws=self.ws,
+                           out=self.idx)
+
+    def attend(self):
+        self.vx.sparse_attn_fwd(self.q, self.k, self.v, self.idx, self.s.T, out=self.o,
+                                lse=self.lse, status=self.status)
+
+    def dense(self):
+        self.vx.sparse_attn_fwd(self.q, self.k, self.v, None, self.s.T, out=self.o_dense,
+                                want_lse=False, status=self.status)
+
+    def step(self, ev=None):
+        if ev is None:
+            self.geometry()
+            self.route()
+            self.attend()
+            return
+        ev[0].record()
+        self.geometry()
+        ev[1].record()
+        self.route()
+        ev[2].record()
+        self.attend()
+        ev[3].record()
+
+
+def time_loop(torch, fn, reps):
+    st = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(st)
+    for _ in range(reps):
+        fn()
+    b.record(st)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+
+    cfg = 4 if args.workload == "sweep" else 3
+    case = synth.make_case(cfg, seed=1000 + cfg + rank, P=args.P)
+    s = case.shape
+    w = Workload(case, device)
+    peaks, peak_kind = load_peaks()
+
+    # warm-up (also the first-call costs: tensor-map encode, attribute set)
+    for _ in range(max(3, args.warmup)):
+        w.step()
+    w.dense()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K whole steps, with per-stage events
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_start.record()
+        for i in range(args.steps):
+            w.step(evs[i])
+        t_end.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    clocks = clk.summary()
+    ms_total = t_start.elapsed_time(t_end)
+    geo_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    route_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    status = int(w.status.item())
+
+    # ---- dense baseline, timed alone (inputs > L2, so no flush is needed)
+    dense_reps = max(3, min(20, args.steps // 10))
+    dense_ms = time_loop(torch, w.dense, dense_reps)
+
+    # ---- end to end through the public API with host buffers: each step copies
+    # the chunk's new inputs (Q, the current chunk's K and V, its depth map and
+    # camera) from pinned host memory and reads O back
+    h_q = w.q.cpu().pin_memory()
+    h_k = w.k[:, :, s.P * s.Nq:].contiguous().cpu().pin_memory()
+    h_v = w.v[:, :, s.P * s.Nq:].contiguous().cpu().pin_memory()
+    h_depth = w.cur_depth.cpu().pin_memory()
+    h_cam = w.cur_cam.cpu().pin_memory()
+    h_o = torch.empty(w.o.shape, dtype=w.o.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_depth, h_cam))
+    d2h = h_o.numel() * h_o.element_size()
+
+    def e2e_step():
+        w.q.copy_(h_q, non_blocking=True)
+        w.k[:, :, s.P * s.Nq:].copy_(h_k, non_blocking=True)
+        w.v[:, :, s.P * s.Nq:].copy_(h_v, non_blocking=True)
+        w.cur_depth.copy_(h_depth, non_blocking=True)
+        w.cur_cam.copy_(h_cam, non_blocking=True)
+        w.step()
+        h_o.copy_(w.o, non_blocking=True)
+
+    e2e_reps = max(3, min(50, args.steps // 4))
+    for _ in range(2):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    e2e_ms = time_loop(torch, e2e_step, e2e_reps)
+
+    # ---- max over ranks
+    vals = torch.tensor([ms_total, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_total, e2e_ms = vals.tolist()
+    ms_step = ms_total / args.steps
+
+    kf, df = kept_flops(s), dense_flops(s)
+    value = world * kf / (ms_step * 1e-3) / 1e12
+    attn_tflops = kf / (attn_ms * 1e-3) / 1e12
+    rbytes = routing_bytes(s)
+    route_gbs = rbytes / (route_ms * 1e-3) / 1e9
+    peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    out = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": workload_desc(s),
+            "l2": "inputs larger than L2 (past K and V are 1.39 GB each at chunk 48); no flush",
+            "kept_fraction": round(s.topk / s.nKB, 4),
+            "parallelism": f"replicated chunks x{world} (one per GPU, no collective)",
+        },
+        "routed_attn_ms": round(attn_ms, 4),
+        "routing_ms": round(route_ms, 4),
+        "geometry_ms": round(geo_ms, 4),
+        "dense_attn_ms": round(dense_ms, 4),
+        "attn_tflops_kept": round(attn_tflops, 2),
+        "dense_tflops": round(df / (dense_ms * 1e-3) / 1e12, 2),
+        "routing_gbs": round(route_gbs, 1),
+        "routing_hbm_frac": round(route_gbs / peaks["hbm_gbs"], 4),
+        "speedup_vs_dense": round(dense_ms / (route_ms + attn_ms), 3),
+        "attn_speedup_vs_dense": round(dense_ms / attn_ms, 3),
+        "allowed_speedup": round(s.nKB / s.topk, 3),
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "attn_fwd_kernel<128,128> (sparse, kept blocks)",
+            "achieved": round(attn_tflops, 2),
+            "peak": peak_t,
+            "peak_kind": f"bf16 sustained ({peak_kind})",
+            "unit": "TFLOP/s",
+            "frac": round(attn_tflops / peak_t, 4),
+            "traffic": None,
+        },
+        "routing_roofline": {
+            "bound": "hbm", "achieved": round(route_gbs, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(route_gbs / peaks["hbm_gbs"], 4),
+            "algorithmic_bytes": rbytes,
+        },
+        "e2e": {
+            "value": round(world * kf / (e2e_ms * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s",
+            "ms_per_step": round(e2e_ms, 4),
+            "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h),
+            "note": "past KV cache resident; per step the chunk's Q/K/V, depth and camera go "
+                    "host->device and O comes back",
+        },
+        "gpu_launches": w.launches_per_step * args.steps,
+        "device_status": status,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        est, took, desc = oracle_sample(case)
+        out["cpu_baseline"] = {
+            "value": round(kf / est / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_threads(),
+            "kind": "oracle", "sample": desc, "sample_seconds": round(took, 2),
+            "est_step_seconds": round(est, 2),
+        }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    cfg = 4 if args.workload == "sweep" else 3
+    case = synth.make_case(cfg, seed=1000 + cfg, P=args.P, heads=(0,))
+    s = synth.shape_for(cfg, P=args.P)
+    case.shape = s
+    kf = kept_flops(s)
+    # rows per step sized so that warm-up + K steps stay within a few minutes
+    n_rows = max(1, min(s.m, (3 * s.m) // max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(case, n_rows=n_rows)
+    ests, took = [], 0.0
+    for _ in range(args.steps):
+        est, t, desc = oracle_sample(case, n_rows=n_rows)
+        ests.append(est)
+        took += t
+    est = statistics.mean(ests)
+    value = kf / est / 1e12
+    out = {
+        "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": workload_desc(s), "l2": "n/a (host)",
+                   "parallelism": "host cores, rank 0 only"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
+    ap.add_argument("--workload", default="headline", choices=["headline", "sweep"])
+    ap.add_argument("--P", type=int, default=None, help="past chunks (sweep workload)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

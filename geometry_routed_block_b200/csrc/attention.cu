@@ -1,0 +1,435 @@
+// Block-sparse attention forward for sm_100a over routed key blocks.
+//
+// Method: "Velox: Raumgedaechtnis beschleunigt Video-Weltmodelle", section
+// "Tiefenanalyse" -- the router decides at the granularity of the kernel's
+// tile, so the kernel really skips the key blocks it is not given. Here one
+// CTA owns a 128-row query tile of one (batch, head) and walks only the key
+// blocks listed for its query block.
+//
+// CTA = 6 warps:
+//   warps 0-3  softmax / correction / epilogue; thread i owns query row i,
+//              which is TMEM lane i
+//   warp 4     TMA producer: Q once, then K_j and V_j of every listed block
+//              (128-byte swizzled tiles, no multicast)
+//   warp 5     tcgen05 issuer (one thread): S_j = Q K_j^T into a double-buffered
+//              TMEM S, O += P_j V_j into TMEM O
+// Tensor memory: S[2] (BN fp32 columns each) and O (D fp32 columns).
+// Online softmax in fp32, base-2 exponent; the running max is only raised
+// when a row's max grows by more than 2^8, so O is rescaled rarely; the final
+// normalisation divides by the running sum taken with the same max.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "ptx.cuh"
+#include "velox_internal.cuh"
+
+namespace velox {
+
+namespace {
+
+constexpr int BM = 128;          // query rows per CTA tile (MMA M)
+constexpr int NTHREADS = 192;    // 6 warps
+constexpr int STAGES = 2;        // K and V ring depth
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any legitimate wait
+constexpr float RESCALE_THRESHOLD = 8.0f;          // log2 units
+
+template <int D, int BN>
+struct Layout {
+    static constexpr int Q_BYTES = BM * D * 2;
+    static constexpr int KV_TILE = BN * D * 2;
+    static constexpr int P_BYTES = BM * BN * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
+    static constexpr int OFF_P = OFF_V + STAGES * KV_TILE;
+    static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+    // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_empty[2], p_full[2], pv_done[2]
+    static constexpr int NBAR = 1 + 4 * STAGES + 8;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
+    static constexpr int TMEM_S = 0;
+    static constexpr int TMEM_O = 2 * BN;
+    static constexpr int TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct Bars {
+    uint32_t base;
+    __device__ uint32_t q_full() const { return base; }
+    __device__ uint32_t k_full(int s) const { return base + 8 * (1 + s); }
+    __device__ uint32_t k_empty(int s) const { return base + 8 * (1 + STAGES + s); }
+    __device__ uint32_t v_full(int s) const { return base + 8 * (1 + 2 * STAGES + s); }
+    __device__ uint32_t v_empty(int s) const { return base + 8 * (1 + 3 * STAGES + s); }
+    __device__ uint32_t s_full(int i) const { return base + 8 * (1 + 4 * STAGES + i); }
+    __device__ uint32_t s_empty(int i) const { return base + 8 * (3 + 4 * STAGES + i); }
+    __device__ uint32_t p_full(int i) const { return base + 8 * (5 + 4 * STAGES + i); }
+    __device__ uint32_t pv_done(int i) const { return base + 8 * (7 + 4 * STAGES + i); }
+};
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+// bounded wait, made uniform across the warp (a warp leaves together)
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+    bool ok = mbar_wait(bar, parity, abort, WAIT_LIMIT_NS);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
+    // waits for copies already in flight; ignores the abort flag, short limit
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > 100000000ull) return false;
+    }
+    return true;
+}
+
+template <int D, int BN>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+    using L = Layout<D, BN>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (sbase - raw);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int qb = blockIdx.x;
+    const int bh = blockIdx.z * a.H + blockIdx.y;
+    const int n = a.n_sel;
+
+    Bars bars{sbase + L::OFF_BAR};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bars.q_full(), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bars.k_full(s), 1);
+            mbar_init(bars.k_empty(s), 1);
+            mbar_init(bars.v_full(s), 1);
+            mbar_init(bars.v_empty(s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bars.s_full(i), 1);
+            mbar_init(bars.s_empty(i), 128);
+            mbar_init(bars.p_full(i), 128);
+            mbar_init(bars.pv_done(i), 1);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const int qrow0 = bh * a.Nq + qb * a.T;
+            const int krow0 = bh * a.Nk;
+            mbar_arrive_expect_tx(bars.q_full(), L::Q_BYTES);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+                tma_load_2d(sbase + L::OFF_Q + c * (BM * 128), &tmQ, bars.q_full(), c * 64, qrow0);
+            const int32_t* row_idx =
+                a.idx ? a.idx + (static_cast<size_t>(bh) * a.m + qb) * static_cast<size_t>(n)
+                      : nullptr;
+            auto fetch = [&](int j) -> int {
+                int kb = row_idx ? __ldg(row_idx + j) : j;
+                if (kb < 0 || kb >= a.n_kb) {
+                    if (a.status) atomicOr(a.status, VELOX_STATUS_BAD_INDEX);
+                    kb = 0;
+                }
+                return kb;
+            };
+            int kb = fetch(0);
+            int issued = 0;
+            for (int j = 0; j < n; ++j) {
+                const int s = j % STAGES;
+                const uint32_t par = ((j / STAGES) - 1) & 1;
+                const int kb_next = (j + 1 < n) ? fetch(j + 1) : 0;
+                const int krow = krow0 + kb * BN;
+                if (j >= STAGES && !mbar_wait(bars.k_empty(s), par, abort_flag, WAIT_LIMIT_NS)) break;
+                mbar_arrive_expect_tx(bars.k_full(s), L::KV_TILE);
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_2d(sbase + L::OFF_K + s * L::KV_TILE + c * (BN * 128), &tmK,
+                                bars.k_full(s), c * 64, krow);
+                if (j >= STAGES && !mbar_wait(bars.v_empty(s), par, abort_flag, WAIT_LIMIT_NS)) {
+                    issued = 2 * j + 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(bars.v_full(s), L::KV_TILE);
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_2d(sbase + L::OFF_V + s * L::KV_TILE + c * (BN * 128), &tmV,
+                                bars.v_full(s), c * 64, krow);
+                issued = 2 * j + 2;
+                kb = kb_next;
+            }
+            // Copies still in flight (only possible after an abort) must land
+            // before the CTA exits: wait for the last ones of every slot.
+            drain_wait(bars.q_full(), 0);
+            for (int t = issued - 1; t >= 0 && t >= issued - 2 * STAGES; --t) {
+                const int j = t >> 1, s = j % STAGES;
+                const uint32_t par = (j / STAGES) & 1;
+                drain_wait((t & 1) ? bars.v_full(s) : bars.k_full(s), par);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t ID_S = idesc_bf16_f32(BM, BN, false, false);
+            constexpr uint32_t ID_PV = idesc_bf16_f32(BM, D, false, true);
+            bool ok = mbar_wait(bars.q_full(), 0, abort_flag, WAIT_LIMIT_NS);
+            tc_fence_after();
+            auto issue_s = [&](int j) -> bool {
+                const int s = j % STAGES;
+                const int bi = j & 1;
+                if (!mbar_wait(bars.k_full(s), (j / STAGES) & 1, abort_flag, WAIT_LIMIT_NS))
+                    return false;
+                if (j >= 2 &&
+                    !mbar_wait(bars.s_empty(bi), ((j >> 1) - 1) & 1, abort_flag, WAIT_LIMIT_NS))
+                    return false;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + L::TMEM_S + bi * BN;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk & 3) * 32;  // 16 bf16 along K inside a 128-B row
+                    const uint64_t ad =
+                        smem_desc_sw128(sbase + L::OFF_Q + (kk >> 2) * (BM * 128) + off, 16);
+                    const uint64_t bd = smem_desc_sw128(
+                        sbase + L::OFF_K + s * L::KV_TILE + (kk >> 2) * (BN * 128) + off, 16);
+                    mma_bf16_ss(d_tmem, ad, bd, ID_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bars.k_empty(s));
+                mma_commit(bars.s_full(bi));
+                return true;
+            };
+            if (ok && n > 0) ok = issue_s(0);
+            for (int j = 0; ok && j < n; ++j) {
+                if (j + 1 < n && !issue_s(j + 1)) break;
+                const int s = j % STAGES;
+                const int bi = j & 1;
+                if (!mbar_wait(bars.v_full(s), (j / STAGES) & 1, abort_flag, WAIT_LIMIT_NS)) break;
+                if (!mbar_wait(bars.p_full(bi), (j >> 1) & 1, abort_flag, WAIT_LIMIT_NS)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(
+                        sbase + L::OFF_P + bi * L::P_BYTES + (kk >> 2) * (BM * 128) + (kk & 3) * 32,
+                        16);
+                    const uint64_t bd = smem_desc_sw128(
+                        sbase + L::OFF_V + s * L::KV_TILE + kk * (16 * 128), BN * 128);
+                    mma_bf16_ss(tmem + L::TMEM_O, ad, bd, ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bars.v_empty(s));
+                mma_commit(bars.pv_done(bi));
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroup
+        const int row = threadIdx.x;  // 0..127
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t t_o = tmem + lane_base + L::TMEM_O;
+        const float sl2 = a.scale_log2;
+        float m_run = -INFINITY;
+        float l_run = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n; ++j) {
+            const int bi = j & 1;
+            if (!warp_wait(bars.s_full(bi), (j >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float s[BN];
+            const uint32_t t_s = tmem + lane_base + L::TMEM_S + bi * BN;
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_s + c * 32, s + c * 32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) reg_fence32(s + c * 32);
+            tc_fence_before();
+            mbar_arrive(bars.s_empty(bi));
+
+            float mx = s[0];
+#pragma unroll
+            for (int i = 1; i < BN; ++i) mx = fmaxf(mx, s[i]);
+            mx *= sl2;
+            float m_new = m_run;
+            bool resc = false;
+            if (mx > m_run + RESCALE_THRESHOLD) {
+                m_new = mx;
+                resc = (j > 0);
+            }
+            const float neg = -m_new;
+            float rs = 0.f;
+#pragma unroll
+            for (int i = 0; i < BN; ++i) {
+                s[i] = ex2_approx(fmaf(s[i], sl2, neg));
+                rs += s[i];
+            }
+            // P buffer bi was last read by PV_{j-2}
+            if (j >= 2 && !warp_wait(bars.pv_done(bi), ((j - 2) >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const uint32_t p_row = sbase + L::OFF_P + bi * L::P_BYTES + row * 128;
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float* p = s + c * 64 + u * 8;
+                    st_shared_v4(p_row + c * (BM * 128) + ((u ^ (row & 7)) << 4),
+                                 pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
+                                 pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+                }
+            }
+            if (__any_sync(0xffffffffu, resc)) {
+                // O must hold PV_{j-1} before it is rescaled
+                if (!warp_wait(bars.pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float f = resc ? ex2_approx(m_run - m_new) : 1.f;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(t_o + c * 32, o);
+                    tmem_wait_ld();
+                    reg_fence32(o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] *= f;
+                    tmem_st32(t_o + c * 32, o);
+                }
+                tmem_wait_st();
+                l_run *= f;
+            }
+            l_run += rs;
+            m_run = m_new;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bars.p_full(bi));
+        }
+        if (ok && n > 0 && warp_wait(bars.pv_done((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag)) {
+            tc_fence_after();
+            const float inv = 1.f / l_run;
+            const bool store = row < a.T;
+            const size_t grow = static_cast<size_t>(bh) * a.Nq + static_cast<size_t>(qb) * a.T + row;
+            __nv_bfloat16* orow = a.o + grow * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                float o[32];
+                tmem_ld32(t_o + c * 32, o);
+                tmem_wait_ld();
+                reg_fence32(o);
+                if (store) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float* p = o + u * 8;
+                        dst[u] = make_uint4(pack_bf16x2(p[0] * inv, p[1] * inv),
+                                            pack_bf16x2(p[2] * inv, p[3] * inv),
+                                            pack_bf16x2(p[4] * inv, p[5] * inv),
+                                            pack_bf16x2(p[6] * inv, p[7] * inv));
+                    }
+                }
+            }
+            if (store && a.lse) a.lse[grow] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+        }
+    }
+
+    if (threadIdx.x == 0 && *abort_flag && a.status) atomicOr(a.status, VELOX_STATUS_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag flag;
+    std::call_once(flag, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// rows x cols bf16 matrix (row-major), boxes of box_rows x 64 columns, 128-byte swizzle
+bool make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols,
+               uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int BN>
+int launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B,
+           cudaStream_t st) {
+    using L = Layout<D, BN>;
+    CUtensorMap tq, tk, tv;
+    const uint64_t bh = static_cast<uint64_t>(B) * a.H;
+    if (!make_tmap(&tq, q, bh * a.Nq, D, BM) || !make_tmap(&tk, k, bh * a.Nk, D, BN) ||
+        !make_tmap(&tv, v, bh * a.Nk, D, BN))
+        return VELOX_ECUDA;
+    auto kern = attn_fwd_kernel<D, BN>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) !=
+        cudaSuccess)
+        return VELOX_ECUDA;
+    dim3 grid(a.m, a.H, B);
+    kern<<<grid, NTHREADS, L::SMEM, st>>>(tq, tk, tv, a);
+    return cudaGetLastError() == cudaSuccess ? VELOX_OK : VELOX_ECUDA;
+}
+
+}  // namespace
+
+int attn_fwd_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B, int d,
+                    cudaStream_t st) {
+    if (d == 128 && a.T == 128) return launch<128, 128>(q, k, v, a, B, st);
+    if (d == 128 && a.T == 64) return launch<128, 64>(q, k, v, a, B, st);
+    if (d == 64 && a.T == 128) return launch<64, 128>(q, k, v, a, B, st);
+    if (d == 64 && a.T == 64) return launch<64, 64>(q, k, v, a, B, st);
+    return VELOX_EUNSUPPORTED;
+}
+
+}  // namespace velox

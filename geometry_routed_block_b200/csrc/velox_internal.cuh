@@ -1,0 +1,48 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/velox.h"
+
+namespace velox {
+
+struct AttnArgs {
+    const int32_t* idx;  // [B*H][m][n_sel] or nullptr (dense)
+    int n_sel;           // key blocks per query block
+    int H, Nq, Nk, T, m, n_kb;
+    float scale_log2;    // softmax scale * log2(e)
+    __nv_bfloat16* o;
+    float* lse;
+    int32_t* status;
+};
+
+int attn_fwd_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B, int d,
+                    cudaStream_t st);
+
+int slices_launch(const float* depth, const float* poses, const float* intr, int P, int HW,
+                  velox_slice_t* out, cudaStream_t st);
+int overlap_launch(const float* depth, const velox_slice_t* cur, const velox_slice_t* slices, int B,
+                   int P, int Hp, int Wp, int T, int m, int32_t* counts, cudaStream_t st);
+size_t multiwarp_ws_bytes(int HW);
+int multiwarp_launch(const float* past_depth, const velox_slice_t* past, const velox_slice_t* cur,
+                     int P, int Hp, int Wp, float rel_tol, float* out, void* ws, cudaStream_t st);
+
+struct RouteArgs {
+    int B, H, Nq, Nk, d, T, m, P, n_past, topk;
+    const int32_t* counts;
+    float alpha, inv_sqrt_d;
+    int32_t* idx;
+    float* qbar;    // workspace [B*H*m][d]
+    float* scores;  // workspace [B*H*m][n_past]
+};
+size_t route_ws_bytes(int B, int H, int m, int n_past, int d);
+int route_launch(const void* q, const void* k, int dtype, const RouteArgs& r, cudaStream_t st);
+
+int cast_bf16_launch(const float* x, uint16_t* y, size_t n, cudaStream_t st);
+
+}  // namespace velox

@@ -23,6 +23,8 @@ Workloads (sizes from the method's headline chunk-48 setting and its neighbours)
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -314,6 +316,15 @@ def _tiny(seed: int) -> Case:
                 past_cams=np.stack(past)[None], slices_given=True)
 
 
+def _parallel_heads(fn, jobs):
+    """Run per-head generators on a thread pool (numpy releases the GIL)."""
+    workers = max(1, min(32, os.cpu_count() or 1, len(jobs)))
+    if workers == 1:
+        return [fn(*j) for j in jobs]
+    with ThreadPoolExecutor(workers) as ex:
+        return list(ex.map(lambda j: fn(*j), jobs))
+
+
 def _walk(seed: int, s: Shape) -> Case:
     rng = np.random.default_rng(seed)
     scene = ground_scene(rng)
@@ -324,14 +335,17 @@ def _walk(seed: int, s: Shape) -> Case:
     q = np.empty((L, s.B, s.H, s.Nq, s.d), np.uint16)
     k = np.empty((L, s.B, s.H, s.Nk, s.d), np.uint16)
     v = np.empty((L, s.B, s.H, s.Nk, s.d), np.uint16)
-    for l in range(L):
-        for h in range(s.H):
-            q[l, 0, h] = f32_to_bf16_bits(_normal(rng, (s.Nq, s.d)))
-            off = (0.5 * _normal(rng, (s.P, 1, s.d)))
-            kh = _normal(rng, (s.P + 1, s.Nq, s.d))
-            kh[: s.P] += off
-            k[l, 0, h] = f32_to_bf16_bits(kh.reshape(s.Nk, s.d))
-            v[l, 0, h] = f32_to_bf16_bits(_normal(rng, (s.Nk, s.d)))
+
+    def head(l, h):
+        hrng = np.random.default_rng([seed, l, h])
+        q[l, 0, h] = f32_to_bf16_bits(_normal(hrng, (s.Nq, s.d)))
+        off = 0.5 * _normal(hrng, (s.P, 1, s.d))  # one mean offset per past chunk
+        kh = _normal(hrng, (s.P + 1, s.Nq, s.d))
+        kh[: s.P] += off
+        k[l, 0, h] = f32_to_bf16_bits(kh.reshape(s.Nk, s.d))
+        v[l, 0, h] = f32_to_bf16_bits(_normal(hrng, (s.Nk, s.d)))
+
+    _parallel_heads(head, [(l, h) for l in range(L) for h in range(s.H)])
     past_poses = np.stack(poses[: s.P])
     past_intr = np.tile(intr, (s.P, 1))
     cams = np.stack([camera_record(p, intr) for p in poses[: s.P]])
@@ -359,19 +373,18 @@ def _loop(cfg: int, seed: int, s: Shape, heads: tuple | None = None) -> Case:
     q = np.empty((L, s.B, len(hsel), s.Nq, s.d), np.uint16)
     k = np.empty((L, s.B, len(hsel), s.Nk, s.d), np.uint16)
     v = np.empty((L, s.B, len(hsel), s.Nk, s.d), np.uint16)
-    for l in range(L):
-        lrng = np.random.default_rng([seed, l])
-        mu = 0.5 * _normal(lrng, (s.H, s.d))
-        for h in range(s.H):
-            hrng = np.random.default_rng([seed, l, h])
-            if h not in hsel:
-                continue
-            i = hsel.index(h)
-            q[l, 0, i] = f32_to_bf16_bits(_normal(hrng, (s.Nq, s.d)) + mu[h])
-            kh = _normal(hrng, (s.P + 1, s.Nq, s.d))
-            kh[: s.P] += ov[:, None, None] * mu[h][None, None, :]
-            k[l, 0, i] = f32_to_bf16_bits(kh.reshape(s.Nk, s.d))
-            v[l, 0, i] = f32_to_bf16_bits(_normal(hrng, (s.Nk, s.d)))
+    mus = [0.5 * _normal(np.random.default_rng([seed, l]), (s.H, s.d)) for l in range(L)]
+
+    def head(l, i, h):
+        hrng = np.random.default_rng([seed, l, h])
+        mu = mus[l][h]
+        q[l, 0, i] = f32_to_bf16_bits(_normal(hrng, (s.Nq, s.d)) + mu)
+        kh = _normal(hrng, (s.P + 1, s.Nq, s.d))
+        kh[: s.P] += ov[:, None, None] * mu[None, None, :]
+        k[l, 0, i] = f32_to_bf16_bits(kh.reshape(s.Nk, s.d))
+        v[l, 0, i] = f32_to_bf16_bits(_normal(hrng, (s.Nk, s.d)))
+
+    _parallel_heads(head, [(l, i, h) for l in range(L) for i, h in enumerate(hsel)])
     past_poses = np.stack(poses[: s.P])
     cams = np.stack([camera_record(p, intr) for p in poses[: s.P]])
     return Case(cfg=cfg, shape=s, seed=seed, q=q, k=k, v=v, cur_depth=depths[s.P][None],

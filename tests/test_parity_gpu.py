@@ -1,0 +1,288 @@
+"""GPU parity: the CUDA path (through the C ABI binding) against the fp64 CPU
+oracle on the same seeded inputs. Needs a B200 and the built libvelox.so."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from geometry_routed_block_b200 import synth
+from oracle import velox_oracle as vo
+from tests.parity_utils import compare_attention, compare_selection, dev, host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def vx():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from geometry_routed_block_b200 import velox
+    return velox
+
+
+def cams_of(case):
+    return dev(case.past_cams), dev(case.cur_cam)
+
+
+# ---------------------------------------------------------------- workload 1 (tiny, fp32)
+
+@pytest.fixture(scope="module")
+def tiny():
+    return synth.make_case(1)
+
+
+def test_tiny_overlap_counts_exact(vx, tiny):
+    s = tiny.shape
+    past, cur = cams_of(tiny)
+    counts = vx.block_overlap(dev(tiny.cur_depth), cur, past, s.F, s.T)
+    want = vo.block_overlap(tiny.cur_depth, tiny.cur_cam, tiny.past_cams, s.F, s.T)
+    assert np.array_equal(counts.cpu().numpy(), want)
+    assert want.sum() > 0
+
+
+def test_tiny_routing_matches_oracle(vx, tiny):
+    s = tiny.shape
+    counts = vo.block_overlap(tiny.cur_depth, tiny.cur_cam, tiny.past_cams, s.F, s.T)
+    q, k = dev(tiny.q[0]), dev(tiny.k[0])
+    for alpha, topk in ((2.0, 6), (0.0, 6), (2.0, 4), (2.0, 20), (50.0, 11)):
+        idx = vx.route_topk(q, k, dev(counts), alpha, topk, s.T)
+        want, s_mod = vo.route_topk(tiny.q[0], tiny.k[0], counts, alpha, topk, s.T)
+        compare_selection(idx.cpu().numpy(), want, s_mod, s.m)
+    a0 = vx.route_topk(q, k, dev(counts), 0.0, 6, s.T)
+    nat = vx.route_topk(q, k, None, 2.0, 6, s.T)
+    assert torch.equal(a0, nat)  # alpha = 0 is the native routing, bit for bit
+
+
+def test_tiny_cast_matches_host_rounding(vx, tiny):
+    got = host_bits(vx.cast_bf16(dev(tiny.q[0])))
+    assert np.array_equal(got, synth.f32_to_bf16_bits(tiny.q[0]))
+
+
+def test_tiny_attention_sparse_and_dense(vx, tiny):
+    s = tiny.shape
+    counts = vo.block_overlap(tiny.cur_depth, tiny.cur_cam, tiny.past_cams, s.F, s.T)
+    idx, _ = vo.route_topk(tiny.q[0], tiny.k[0], counts, s.alpha, s.topk, s.T)
+    qb, kb, vb = (synth.f32_to_bf16_bits(x[0]) for x in (tiny.q, tiny.k, tiny.v))
+    q, k, v = (vx.cast_bf16(dev(x[0])) for x in (tiny.q, tiny.k, tiny.v))
+    o, lse = vx.sparse_attn_fwd(q, k, v, dev(idx), s.T)
+    o_ref, lse_ref = vo.sparse_attention(qb, kb, vb, idx, s.T)
+    compare_attention(o, o_ref, "tiny sparse")
+    assert np.abs(lse.cpu().numpy() - lse_ref).max() < 1e-3
+    o, lse = vx.sparse_attn_fwd(q, k, v, None, s.T)
+    o_ref, lse_ref = vo.sparse_attention(qb, kb, vb, None, s.T)
+    compare_attention(o, o_ref, "tiny dense")
+    assert np.abs(lse.cpu().numpy() - lse_ref).max() < 1e-3
+
+
+# ---------------------------------------------------------------- workload 2 (dense parity)
+
+@pytest.fixture(scope="module")
+def walk():
+    return synth.make_case(2)
+
+
+def test_walk_slices_and_counts_exact(vx, walk):
+    s = walk.shape
+    sl = vx.slices_build(dev(walk.past_depth[0]), dev(walk.past_poses[0]), dev(walk.past_intr[0]))
+    want_sl = vo.slices_build(walk.past_depth[0], walk.past_poses[0], walk.past_intr[0])
+    assert np.array_equal(sl.cpu().numpy(), want_sl)
+    counts = vx.block_overlap(dev(walk.cur_depth), dev(walk.cur_cam), sl[None], s.F, s.T)
+    want = vo.block_overlap(walk.cur_depth, walk.cur_cam, want_sl[None], s.F, s.T)
+    assert np.array_equal(counts.cpu().numpy(), want)
+    assert want.sum() > 0 and (want < s.T).any()
+
+
+def test_walk_dense_attention_rows(vx, walk):
+    s = walk.shape
+    q, k, v = dev(walk.q[0]), dev(walk.k[0]), dev(walk.v[0])
+    rows = [(0, h, qb) for h in (0, 5, 11) for qb in (0, 17, 35)]
+    ref = vo.sparse_attention(walk.q[0], walk.k[0], walk.v[0], None, s.T, rows=rows)
+    o, lse = vx.sparse_attn_fwd(q, k, v, None, s.T)
+    # top-k = every block, listed explicitly, is the same computation
+    all_idx = torch.arange(s.nKB, dtype=torch.int32, device="cuda").expand(s.B, s.H, s.m, s.nKB)
+    o2, _ = vx.sparse_attn_fwd(q, k, v, all_idx.contiguous(), s.T)
+    for (b, h, qb), (o_ref, lse_ref) in ref.items():
+        sl = slice(qb * s.T, (qb + 1) * s.T)
+        compare_attention(o[b, h, sl], o_ref, f"dense row {(b, h, qb)}")
+        compare_attention(o2[b, h, sl], o_ref, f"all-listed row {(b, h, qb)}")
+        assert np.abs(lse[b, h, sl].cpu().numpy() - lse_ref).max() < 1e-3
+    assert torch.equal(o, o2)
+
+
+def test_walk_routing_alpha0_and_geometry(vx, walk):
+    s = walk.shape
+    sl = vo.slices_build(walk.past_depth[0], walk.past_poses[0], walk.past_intr[0])
+    counts = vo.block_overlap(walk.cur_depth, walk.cur_cam, sl[None], s.F, s.T)
+    q, k = dev(walk.q[0]), dev(walk.k[0])
+    topk = 65
+    total_ties = 0
+    for alpha, cnt in ((0.0, counts), (2.0, counts), (2.0, None)):
+        idx = vx.route_topk(q, k, None if cnt is None else dev(cnt), alpha, topk, s.T)
+        want, s_mod = vo.route_topk(walk.q[0], walk.k[0], cnt, alpha, topk, s.T)
+        total_ties += compare_selection(idx.cpu().numpy(), want, s_mod, s.m)
+    assert total_ties <= 3
+
+
+def test_walk_routed_attention(vx, walk):
+    s = walk.shape
+    sl = vo.slices_build(walk.past_depth[0], walk.past_poses[0], walk.past_intr[0])
+    counts = vo.block_overlap(walk.cur_depth, walk.cur_cam, sl[None], s.F, s.T)
+    idx, _ = vo.route_topk(walk.q[0], walk.k[0], counts, s.alpha, 65, s.T)
+    rows = [(0, h, qb) for h in (1, 7) for qb in (0, 9, 35)]
+    ref = vo.sparse_attention(walk.q[0], walk.k[0], walk.v[0], idx, s.T, rows=rows)
+    o, _ = vx.sparse_attn_fwd(dev(walk.q[0]), dev(walk.k[0]), dev(walk.v[0]), dev(idx), s.T)
+    for (b, h, qb), (o_ref, _) in ref.items():
+        compare_attention(o[b, h, qb * s.T:(qb + 1) * s.T], o_ref, f"routed row {(b, h, qb)}")
+
+
+# ---------------------------------------------------------------- kernel variants and edges
+
+def _random_qkv(rng, B, H, Nq, Nk, d):
+    f = lambda *sh: synth.f32_to_bf16_bits(rng.standard_normal(sh, dtype=np.float32))
+    return f(B, H, Nq, d), f(B, H, Nk, d), f(B, H, Nk, d)
+
+
+@pytest.mark.parametrize("T,d", [(64, 64), (64, 128), (128, 64), (128, 128)])
+def test_attention_variants_with_duplicates_and_ragged_tiles(vx, T, d):
+    rng = np.random.default_rng(T * 1000 + d)
+    B, H = 2, 3
+    Nq = 3 * T          # three query blocks: for T=64 the last 128-row tile is half outside
+    Nk = 11 * T
+    q, k, v = _random_qkv(rng, B, H, Nq, Nk, d)
+    m, nkb = Nq // T, Nk // T
+    topk = 5
+    idx = rng.integers(0, nkb, size=(B, H, m, topk)).astype(np.int32)
+    idx[0, 0, 0] = [3, 3, 3, 7, 0]   # a block listed several times counts several times
+    o, lse = vx.sparse_attn_fwd(dev(q), dev(k), dev(v), dev(idx), T)
+    o_ref, lse_ref = vo.sparse_attention(q, k, v, idx, T)
+    compare_attention(o, o_ref, f"T={T} d={d}")
+    assert np.abs(lse.cpu().numpy() - lse_ref).max() < 1e-3
+    o, _ = vx.sparse_attn_fwd(dev(q), dev(k), dev(v), None, T)
+    o_ref, _ = vo.sparse_attention(q, k, v, None, T)
+    compare_attention(o, o_ref, f"dense T={T} d={d}")
+
+
+def test_attention_large_logits_rescale(vx):
+    # scores that grow along the walk force the running max (and O) to be rescaled
+    rng = np.random.default_rng(7)
+    T, d, B, H = 128, 128, 1, 2
+    Nq, Nk = 256, 2048
+    qf = rng.standard_normal((B, H, Nq, d), dtype=np.float32)
+    kf = rng.standard_normal((B, H, Nk, d), dtype=np.float32)
+    ramp = np.linspace(0.2, 6.0, Nk, dtype=np.float32)[None, None, :, None]
+    kf = kf * ramp + ramp * qf.mean(axis=2, keepdims=True)
+    q, k = synth.f32_to_bf16_bits(qf), synth.f32_to_bf16_bits(kf)
+    v = synth.f32_to_bf16_bits(rng.standard_normal((B, H, Nk, d), dtype=np.float32))
+    o, lse = vx.sparse_attn_fwd(dev(q), dev(k), dev(v), None, T)
+    o_ref, lse_ref = vo.sparse_attention(q, k, v, None, T)
+    compare_attention(o, o_ref, "rescale")
+    assert np.abs(lse.cpu().numpy() - lse_ref).max() < 2e-3
+
+
+def test_route_topk_extremes(vx, walk):
+    s = walk.shape
+    q, k = dev(walk.q[0]), dev(walk.k[0])
+    only_cur = vx.route_topk(q, k, None, 0.0, s.m, s.T).cpu().numpy()
+    assert (only_cur == np.arange(s.nKB - s.m, s.nKB)).all()
+    everything = vx.route_topk(q, k, None, 0.0, s.nKB, s.T).cpu().numpy()
+    assert (everything == np.arange(s.nKB)).all()
+
+
+def test_bad_indices_are_flagged_not_faulting(vx):
+    rng = np.random.default_rng(11)
+    T, d = 128, 128
+    q, k, v = _random_qkv(rng, 1, 1, 256, 1024, d)
+    idx = np.array([[[[0, 1, -5], [2, 8, 3]]]], dtype=np.int32)  # -5 and 8 are out of range
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, _ = vx.sparse_attn_fwd(dev(q), dev(k), dev(v), dev(idx), T, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & vx.VELOX_STATUS_BAD_INDEX
+    assert torch.isfinite(o.float()).all()
+    fixed = np.array([[[[0, 1, 0], [2, 0, 3]]]], dtype=np.int32)  # replaced by block 0
+    o_ref, _ = vo.sparse_attention(q, k, v, fixed, T)
+    compare_attention(o, o_ref, "bad-index replacement")
+    status.zero_()
+    vx.sparse_attn_fwd(dev(q), dev(k), dev(v), dev(fixed), T, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+
+# ---------------------------------------------------------------- multiwarp
+
+def test_multiwarp_hand_example(vx):
+    from tests.test_oracle_pins import read_fixture
+    g = read_fixture("multiwarp_worked.txt")
+    Hp, Wp, rel = int(g["Hp Wp rel_tol"][0]), int(g["Hp Wp rel_tol"][1]), g["Hp Wp rel_tol"][2]
+    cam = np.array(g["cam"], dtype=np.float32)
+    d = np.stack([np.array(g["depth_chunk0"], np.float32),
+                  np.array(g["depth_chunk1"], np.float32)]).reshape(2, Hp, Wp)
+    out = vx.depth_multiwarp(dev(d), dev(np.stack([cam, cam])), dev(cam), rel)
+    assert np.array_equal(out.cpu().numpy(), np.array(g["expected"], np.float32).reshape(Hp, Wp))
+
+
+def test_multiwarp_pipeline_geometry_exact(vx):
+    c = synth.geometry_only(5)
+    s = c.shape
+    cams = np.stack([synth.camera_record(c.past_poses[0, j], c.past_intr[0, j]) for j in range(s.P)])
+    got = vx.depth_multiwarp(dev(c.past_depth[0]), dev(cams), dev(c.cur_cam[0]), 0.01).cpu().numpy()
+    want = vo.depth_multiwarp(c.past_depth[0], cams, c.cur_cam[0], 0.01)
+    assert np.array_equal(got, want, equal_nan=True)
+    assert np.isfinite(want).mean() > 0.5
+    # the warped depth then feeds the overlap counts
+    sl = vo.slices_build(c.past_depth[0], c.past_poses[0], c.past_intr[0])
+    counts = vx.block_overlap(dev(want[None]), dev(c.cur_cam), dev(sl[None]), s.F, s.T)
+    assert np.array_equal(counts.cpu().numpy(), vo.block_overlap(want[None], c.cur_cam, sl[None], s.F, s.T))
+
+
+# ---------------------------------------------------------------- chunk-48 headline, full size
+
+@pytest.fixture(scope="module")
+def headline():
+    return synth.make_case(3)
+
+
+def test_headline_geometry_exact(vx, headline):
+    c = headline
+    s = c.shape
+    sl = vx.slices_build(dev(c.past_depth[0]), dev(c.past_poses[0]), dev(c.past_intr[0]))
+    want_sl = vo.slices_build(c.past_depth[0], c.past_poses[0], c.past_intr[0])
+    assert np.array_equal(sl.cpu().numpy(), want_sl)
+    counts = vx.block_overlap(dev(c.cur_depth), dev(c.cur_cam), sl[None], s.F, s.T)
+    assert np.array_equal(counts.cpu().numpy(),
+                          vo.block_overlap(c.cur_depth, c.cur_cam, want_sl[None], s.F, s.T))
+
+
+def test_headline_routing_and_attention_sampled(vx, headline):
+    c = headline
+    s = c.shape
+    sl = vo.slices_build(c.past_depth[0], c.past_poses[0], c.past_intr[0])
+    counts = vo.block_overlap(c.cur_depth, c.cur_cam, sl[None], s.F, s.T)
+    q, k, v = dev(c.q[0]), dev(c.k[0]), dev(c.v[0])
+    idx = vx.route_topk(q, k, dev(counts), s.alpha, s.topk, s.T)
+    heads = [0, 13, 23]
+    want, s_mod = vo.route_topk(c.q[0][:, heads], c.k[0][:, heads], counts, s.alpha, s.topk, s.T)
+    ties = compare_selection(idx[:, heads].cpu().numpy(), want, s_mod, s.m)
+    assert ties <= 3
+    kept = idx.cpu().numpy()
+    assert kept.shape == (1, s.H, s.m, s.topk)
+    # attention on the oracle's own selection, sampled rows
+    o, lse = vx.sparse_attn_fwd(q, k, v, idx, s.T)
+    rows = [(0, heads[i], qb) for i in range(3) for qb in (0, 20, 35)]
+    ref = vo.sparse_attention(c.q[0][:, heads], c.k[0][:, heads], c.v[0][:, heads], want, s.T,
+                              rows=[(0, i, qb) for i in range(3) for qb in (0, 20, 35)])
+    for (b, h, qb), ((_, i, _), (o_ref, lse_ref)) in zip(rows, ref.items()):
+        if not np.array_equal(kept[0, h, qb], want[0, i, qb]):
+            continue  # a near-tie row: the two selections legitimately differ
+        sl_ = slice(qb * s.T, (qb + 1) * s.T)
+        compare_attention(o[b, h, sl_], o_ref, f"headline row {(b, h, qb)}")
+        assert np.abs(lse[b, h, sl_].cpu().numpy() - lse_ref).max() < 1e-3
+
+
+def test_rollout_p96_routing_sampled_heads(vx):
+    c = synth.make_case(4, P=96, heads=(0, 11))
+    s = c.shape
+    sl = vo.slices_build(c.past_depth[0], c.past_poses[0], c.past_intr[0])
+    counts = vo.block_overlap(c.cur_depth, c.cur_cam, sl[None], s.F, s.T)
+    idx = vx.route_topk(dev(c.q[0]), dev(c.k[0]), dev(counts), s.alpha, s.topk, s.T)
+    want, s_mod = vo.route_topk(c.q[0], c.k[0], counts, s.alpha, s.topk, s.T)
+    assert compare_selection(idx.cpu().numpy(), want, s_mod, s.m) <= 3
