@@ -304,3 +304,59 @@ int cast_bf16_launch(const float* x, uint16_t* y, size_t n, cudaStream_t st) {
 }
 
 }  // namespace velox
+
+// ---------------------------------------------------------------- multiwarp, library-owned scratch
+//
+// Some callers cannot allocate device memory: a plugin whose host hands it
+// only its input and output buffers, or a latency-critical loop that must not
+// call cudaMalloc (which can synchronise the device). For them the multiwarp's
+// per-pixel scratch lives in a fixed array in this library's own device
+// memory. Each GPU that loads the library holds the array until the process
+// exits. All calls share it, so calls that overlap on the GPU race.
+
+#include <mutex>
+
+namespace velox {
+namespace {
+
+constexpr int NOALLOC_MAX_PIXELS = VELOX_MULTIWARP_NOALLOC_MAX_PIXELS;
+constexpr size_t NOALLOC_BYTES =
+    2 * static_cast<size_t>(NOALLOC_MAX_PIXELS) * 8 + static_cast<size_t>(NOALLOC_MAX_PIXELS) * 4;
+constexpr int NOALLOC_MAX_DEVICES = 64;
+
+static __device__ __align__(256) unsigned char g_multiwarp_scratch[NOALLOC_BYTES];
+
+// Device address of the array on the current device. The host-side symbol is
+// only a stand-in; the real address is looked up once per device, with that
+// device current, and cached.
+void* multiwarp_scratch_on_current_device() {
+    static std::mutex mu;
+    static void* addr[NOALLOC_MAX_DEVICES] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_multiwarp_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+}  // namespace velox
+
+extern "C" int velox_depth_multiwarp_noalloc(const float* past_depth,
+                                             const velox_slice_t* past_cams,
+                                             const velox_slice_t* cur_cam, int P, int Hp, int Wp,
+                                             float rel_tol, float* cur_depth, void* stream) {
+    if (!past_depth || !past_cams || !cur_cam || !cur_depth) return VELOX_EINVAL;
+    if (P < 1 || Hp < 1 || Wp < 1 || !(rel_tol >= 0.0f) || !isfinite(rel_tol)) return VELOX_EINVAL;
+    if (static_cast<long long>(Hp) * Wp > velox::NOALLOC_MAX_PIXELS) return VELOX_EINVAL;
+    if (static_cast<long long>(P) * Hp * Wp >= (1ll << 31)) return VELOX_EINVAL;
+    void* scratch = velox::multiwarp_scratch_on_current_device();
+    if (scratch == nullptr) return VELOX_ECUDA;
+    // the launch sequence starts by resetting the per-pixel state it uses
+    return velox::multiwarp_launch(past_depth, past_cams, cur_cam, P, Hp, Wp, rel_tol, cur_depth,
+                                   scratch, static_cast<cudaStream_t>(stream));
+}

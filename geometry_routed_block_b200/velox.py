@@ -49,6 +49,8 @@ SIGNATURES = {
     "velox_depth_multiwarp": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_float, _vp, _vp,
                                        _c_size, _vp]),
     "velox_cast_bf16": (_c_int, [_vp, _vp, _c_size, _vp]),
+    "velox_depth_multiwarp_noalloc": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_float,
+                                               _vp, _vp]),
 }
 
 
@@ -222,4 +224,18 @@ def cast_bf16(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> 
     if out is None:
         out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
     _check(lib.velox_cast_bf16(_ptr(x), _ptr(out), x.numel(), _stream(stream)), "velox_cast_bf16")
+    return out
+
+
+def depth_multiwarp_noalloc(past_depth: torch.Tensor, past_cams: torch.Tensor,
+                            cur_cam: torch.Tensor, rel_tol: float = 0.01,
+                            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """depth_multiwarp with the library's fixed scratch instead of a caller
+    workspace (grids up to 65536 pixels; concurrent calls race)."""
+    P, Hp, Wp = past_depth.shape
+    if out is None:
+        out = torch.empty((Hp, Wp), dtype=torch.float32, device=past_depth.device)
+    _check(lib.velox_depth_multiwarp_noalloc(_ptr(past_depth), _ptr(past_cams), _ptr(cur_cam), P,
+                                             Hp, Wp, float(rel_tol), _ptr(out), _stream(stream)),
+           "velox_depth_multiwarp_noalloc")
     return out

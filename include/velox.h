@@ -197,6 +197,33 @@ VELOX_API int velox_depth_multiwarp(const float* past_depth, const velox_slice_t
                           const velox_slice_t* cur_cam, int P, int Hp, int Wp, float rel_tol,
                           float* cur_depth, void* ws, size_t ws_bytes, void* stream);
 
+/* Largest grid (Hp * Wp) velox_depth_multiwarp_noalloc accepts. */
+#define VELOX_MULTIWARP_NOALLOC_MAX_PIXELS 65536
+
+/*
+ * velox_depth_multiwarp without a caller workspace. The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory -- e.g. a plugin whose host passes it only its input and output
+ * buffers, or a latency-critical loop that must not call cudaMalloc, which can
+ * synchronise the device. Arguments and results are those of
+ * velox_depth_multiwarp, minus ws / ws_bytes. Nothing is allocated or freed:
+ * the scratch (20 bytes per pixel) is a fixed array in the library's own
+ * device memory, 1.25 MiB, held on every GPU that loads the library until the
+ * process exits.
+ *   - Hp * Wp above VELOX_MULTIWARP_NOALLOC_MAX_PIXELS returns VELOX_EINVAL and
+ *     launches nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture. A failed lookup returns VELOX_ECUDA.
+ *   - Every call resets the scratch it uses before reading it, but all calls
+ *     share one array: calls whose kernels overlap on the GPU (e.g. on two
+ *     streams at once) race and give wrong depths. Serialise them.
+ */
+VELOX_API int velox_depth_multiwarp_noalloc(const float* past_depth,
+                                            const velox_slice_t* past_cams,
+                                            const velox_slice_t* cur_cam, int P, int Hp, int Wp,
+                                            float rel_tol, float* cur_depth, void* stream);
+
 /*
  * float32 -> bf16 (round to nearest even) for n elements; used where a
  * workload's Q/K/V arrive in float32 and the attention tiles take bf16.
