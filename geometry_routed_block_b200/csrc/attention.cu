@@ -80,6 +80,29 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// acc[k] = max(acc[k], s[LO + k + 8 i]) over [LO, HI): 8 independent chains,
+// three-input max where possible
+template <int LO, int HI>
+__device__ __forceinline__ void max_range(const float* s, float* acc) {
+    int i = LO;
+#pragma unroll
+    for (; i + 16 <= HI; i += 16) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = max3f(acc[k], s[i + k], s[i + 8 + k]);
+    }
+#pragma unroll
+    for (; i + 8 <= HI; i += 8) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = fmaxf(acc[k], s[i + k]);
+    }
+}
+
 // bounded wait, made uniform across the warp (a warp leaves together)
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
     bool ok = mbar_wait(bar, parity, abort, WAIT_LIMIT_NS);
@@ -126,8 +149,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bars.s_full(i), 1);
-            mbar_init(bars.s_empty(i), 128);
-            mbar_init(bars.p_full(i), 128);
+            mbar_init(bars.s_empty(i), 4);  // one elected arrive per softmax warp
+            mbar_init(bars.p_full(i), 4);
             mbar_init(bars.pv_done(i), 1);
         }
         fence_mbar_init();
@@ -269,17 +292,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_after();
             float s[BN];
             const uint32_t t_s = tmem + lane_base + L::TMEM_S + bi * BN;
+            // first half of the row, then the second half in flight while the
+            // first half is reduced
+            constexpr int HALF = BN / 2;
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_s + c * 32, s + c * 32);
+            for (int c = 0; c < HALF / 32; ++c) tmem_ld32(t_s + c * 32, s + c * 32);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) reg_fence32(s + c * 32);
-            tc_fence_before();
-            mbar_arrive(bars.s_empty(bi));
-
-            float mx = s[0];
+            for (int c = 0; c < HALF / 32; ++c) reg_fence32(s + c * 32);
 #pragma unroll
-            for (int i = 1; i < BN; ++i) mx = fmaxf(mx, s[i]);
+            for (int c = HALF / 32; c < BN / 32; ++c) tmem_ld32(t_s + c * 32, s + c * 32);
+            float acc[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = s[k];
+            max_range<8, HALF>(s, acc);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = HALF / 32; c < BN / 32; ++c) reg_fence32(s + c * 32);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.s_empty(bi));  // S buffer may be overwritten
+            max_range<HALF, BN>(s, acc);
+            float mx = max3f(max3f(acc[0], acc[1], acc[2]), max3f(acc[3], acc[4], acc[5]),
+                             fmaxf(acc[6], acc[7]));
             mx *= sl2;
             float m_new = m_run;
             bool resc = false;
@@ -287,13 +322,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 m_new = mx;
                 resc = (j > 0);
             }
-            const float neg = -m_new;
-            float rs = 0.f;
+            // p = 2^(s * scale * log2e - m), two lanes of fp32 per FFMA2 / FADD2
+            const float2 sc2 = make_float2(sl2, sl2);
+            const float2 ng2 = make_float2(-m_new, -m_new);
+            float2 sum2[4];
 #pragma unroll
-            for (int i = 0; i < BN; ++i) {
-                s[i] = ex2_approx(fmaf(s[i], sl2, neg));
-                rs += s[i];
+            for (int k = 0; k < 4; ++k) sum2[k] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < BN; i += 2) {
+                float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), sc2, ng2);
+                x.x = ex2_approx(x.x);
+                x.y = ex2_approx(x.y);
+                s[i] = x.x;
+                s[i + 1] = x.y;
+                sum2[(i >> 1) & 3] = __fadd2_rn(sum2[(i >> 1) & 3], x);
             }
+            const float2 s01 = __fadd2_rn(sum2[0], sum2[1]);
+            const float2 s23 = __fadd2_rn(sum2[2], sum2[3]);
+            const float2 s03 = __fadd2_rn(s01, s23);
+            const float rs = s03.x + s03.y;
             // P buffer bi was last read by PV_{j-2}
             if (j >= 2 && !warp_wait(bars.pv_done(bi), ((j - 2) >> 1) & 1, abort_flag)) {
                 ok = false;
@@ -335,7 +382,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             m_run = m_new;
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(bars.p_full(bi));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.p_full(bi));  // P_j and (rescaled) O are ready
         }
         if (ok && n > 0 && warp_wait(bars.pv_done((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag)) {
             tc_fence_after();
