@@ -11,9 +11,13 @@
 //              which is TMEM lane i
 //   warp 4     TMA producer: Q once, then K_j and V_j of every listed block
 //              (128-byte swizzled tiles, no multicast)
-//   warp 5     tcgen05 issuer (one thread): S_j = Q K_j^T into a double-buffered
-//              TMEM S, O += P_j V_j into TMEM O
-// Tensor memory: S[2] (BN fp32 columns each) and O (D fp32 columns).
+//   warp 5     tcgen05 issuer (one thread): S_j = Q K_j^T (both operands in
+//              shared memory) into a double-buffered TMEM S; O += P_j V_j with
+//              P_j read from tensor memory and V_j from shared memory
+// Tensor memory: S[2] (BN fp32 columns each), O (D fp32 columns), P[2]
+// (BN/2 columns each: bf16 pairs). Keeping P out of shared memory removes a
+// third of the shared-memory traffic of a tile (both operands of P V and the
+// softmax's P writes would otherwise go through it).
 // Online softmax in fp32, base-2 exponent; the running max is only raised
 // when a row's max grows by more than 2^8, so O is rescaled rarely; the final
 // normalisation divides by the running sum taken with the same max.
@@ -35,7 +39,7 @@ namespace {
 
 constexpr int BM = 128;          // query rows per CTA tile (MMA M)
 constexpr int NTHREADS = 192;    // 6 warps
-constexpr int STAGES = 2;        // K and V ring depth
+constexpr int STAGES = 3;        // K and V ring depth
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr float RESCALE_THRESHOLD = 8.0f;          // log2 units
 
@@ -43,20 +47,21 @@ template <int D, int BN>
 struct Layout {
     static constexpr int Q_BYTES = BM * D * 2;
     static constexpr int KV_TILE = BN * D * 2;
-    static constexpr int P_BYTES = BM * BN * 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
-    static constexpr int OFF_P = OFF_V + STAGES * KV_TILE;
-    static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+    static constexpr int OFF_BAR = OFF_V + STAGES * KV_TILE;
     // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_empty[2], p_full[2], pv_done[2]
     static constexpr int NBAR = 1 + 4 * STAGES + 8;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
+    // tensor memory columns: S[2] (fp32), O (fp32), P[2] (bf16 pairs)
     static constexpr int TMEM_S = 0;
     static constexpr int TMEM_O = 2 * BN;
-    static constexpr int TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+    static constexpr int TMEM_P = 2 * BN + D;
+    static constexpr int TMEM_COLS = (3 * BN + D) <= 256 ? 256 : 512;
+    static_assert(3 * BN + D <= 512, "tensor memory budget");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -263,12 +268,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(
-                        sbase + L::OFF_P + bi * L::P_BYTES + (kk >> 2) * (BM * 128) + (kk & 3) * 32,
-                        16);
+                    // A = P_j from tensor memory: 16 bf16 of a row = 8 columns
+                    const uint32_t at = tmem + L::TMEM_P + bi * (BN / 2) + kk * 8;
                     const uint64_t bd = smem_desc_sw128(
                         sbase + L::OFF_V + s * L::KV_TILE + kk * (16 * 128), BN * 128);
-                    mma_bf16_ss(tmem + L::TMEM_O, ad, bd, ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(tmem + L::TMEM_O, at, bd, ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bars.v_empty(s));
                 mma_commit(bars.pv_done(bi));
@@ -346,16 +350,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 ok = false;
                 break;
             }
-            const uint32_t p_row = sbase + L::OFF_P + bi * L::P_BYTES + row * 128;
+            {
+                // P_j (bf16 pairs, lower key in the low half) into tensor memory
+                float pk[BN / 2];
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c) {
+                for (int i = 0; i < BN / 2; ++i)
+                    pk[i] = __uint_as_float(pack_bf16x2(s[2 * i], s[2 * i + 1]));
+                const uint32_t t_p = tmem + lane_base + L::TMEM_P + bi * (BN / 2);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float* p = s + c * 64 + u * 8;
-                    st_shared_v4(p_row + c * (BM * 128) + ((u ^ (row & 7)) << 4),
-                                 pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
-                                 pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
-                }
+                for (int c = 0; c < BN / 64; ++c) tmem_st32(t_p + c * 32, pk + c * 32);
+                tmem_wait_st();
             }
             if (__any_sync(0xffffffffu, resc)) {
                 // O must hold PV_{j-1} before it is rescaled
@@ -380,7 +384,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             l_run += rs;
             m_run = m_new;
-            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.p_full(bi));  // P_j and (rescaled) O are ready
