@@ -108,6 +108,34 @@ __device__ __forceinline__ void max_range(const float* s, float* acc) {
     }
 }
 
+// 2^x for two lanes on the FMA pipe (Cody-Waite range reduction + minimax
+// cubic; coefficients from geometry_routed_block_b200/exp2_poly.py, relative
+// error < 1e-4). n = round(x) comes from the low mantissa bits of
+// x + 1.5 * 2^23; f = x - n lies in [-1/2, 1/2]; the result is p(f) with n added
+// to its exponent field. x is clamped to [-120, inf): below that 2^x is
+// negligible next to the row sum, and the exponent cannot wrap.
+constexpr float EXP2_C0 = 0.9999280571937561f;
+constexpr float EXP2_C1 = 0.6932609677314758f;
+constexpr float EXP2_C2 = 0.2426111251115799f;
+constexpr float EXP2_C3 = 0.0551716685295105f;
+constexpr unsigned EXP2_EMU_MASK = 0x52;  // pairs 1, 4 and 6 of every 8
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -120.f);
+    x.y = fmaxf(x.y, -120.f);
+    const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
+    const float2 t = __fadd2_rn(x, magic);
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 p = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+    p = __ffma2_rn(p, f, make_float2(EXP2_C1, EXP2_C1));
+    p = __ffma2_rn(p, f, make_float2(EXP2_C0, EXP2_C0));
+    float2 r;
+    r.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
+    r.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
+    return r;
+}
+
 // bounded wait, made uniform across the warp (a warp leaves together)
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
     bool ok = mbar_wait(bar, parity, abort, WAIT_LIMIT_NS);
@@ -326,7 +354,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 m_new = mx;
                 resc = (j > 0);
             }
-            // p = 2^(s * scale * log2e - m), two lanes of fp32 per FFMA2 / FADD2
+            // p = 2^(s * scale * log2e - m), two lanes of fp32 per FFMA2 / FADD2;
+            // the pairs selected by EXP2_EMU_MASK run on the FMA pipe, the rest
+            // on the ex2 unit, so neither pipe alone bounds the loop
             const float2 sc2 = make_float2(sl2, sl2);
             const float2 ng2 = make_float2(-m_new, -m_new);
             float2 sum2[4];
@@ -335,8 +365,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int i = 0; i < BN; i += 2) {
                 float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), sc2, ng2);
-                x.x = ex2_approx(x.x);
-                x.y = ex2_approx(x.y);
+                if ((EXP2_EMU_MASK >> ((i >> 1) & 7)) & 1) {
+                    x = exp2_poly2(x);
+                } else {
+                    x.x = ex2_approx(x.x);
+                    x.y = ex2_approx(x.y);
+                }
                 s[i] = x.x;
                 s[i + 1] = x.y;
                 sum2[(i >> 1) & 3] = __fadd2_rn(sum2[(i >> 1) & 3], x);
