@@ -9,15 +9,15 @@
 // CTA = 6 warps:
 //   warps 0-3  softmax / correction / epilogue; thread i owns query row i,
 //              which is TMEM lane i
-//   warp 4     TMA producer: Q once, then K_j and V_j of every listed block
+//   warp 4     TMA producer: K_j and V_j of every listed block
 //              (128-byte swizzled tiles, no multicast)
-//   warp 5     tcgen05 issuer (one thread): S_j = Q K_j^T (both operands in
-//              shared memory) into a double-buffered TMEM S; O += P_j V_j with
-//              P_j read from tensor memory and V_j from shared memory
-// Tensor memory: S[2] (BN fp32 columns each), O (D fp32 columns), P[2]
-// (BN/2 columns each: bf16 pairs). Keeping P out of shared memory removes a
-// third of the shared-memory traffic of a tile (both operands of P V and the
-// softmax's P writes would otherwise go through it).
+//   warp 5     tcgen05 issuer (one thread): S_j = Q K_j^T into a double-buffered
+//              TMEM S; O += P_j V_j. Q and P_j are A operands read from tensor
+//              memory; only K_j and V_j come from shared memory.
+// Tensor memory: S[2] (BN fp32 columns each), O (D fp32 columns), P (BN/2
+// columns of bf16 pairs), Q (D/2 columns of bf16 pairs; written once by the
+// softmax threads). Keeping Q and P out of shared memory halves the
+// shared-memory traffic of a tile, which otherwise limits the tensor core.
 // Online softmax in fp32, base-2 exponent; the running max is only raised
 // when a row's max grows by more than 2^8, so O is rescaled rarely; the final
 // normalisation divides by the running sum taken with the same max.
@@ -45,10 +45,8 @@ constexpr float RESCALE_THRESHOLD = 8.0f;          // log2 units
 
 template <int D, int BN>
 struct Layout {
-    static constexpr int Q_BYTES = BM * D * 2;
     static constexpr int KV_TILE = BN * D * 2;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
     static constexpr int OFF_BAR = OFF_V + STAGES * KV_TILE;
     // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_empty[2], p_full[2], pv_done[2]
@@ -56,12 +54,14 @@ struct Layout {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
-    // tensor memory columns: S[2] (fp32), O (fp32), P[2] (bf16 pairs)
+    // tensor memory columns: S[2] (fp32), O (fp32), P (bf16 pairs), Q (bf16 pairs)
     static constexpr int TMEM_S = 0;
     static constexpr int TMEM_O = 2 * BN;
     static constexpr int TMEM_P = 2 * BN + D;
-    static constexpr int TMEM_COLS = (3 * BN + D) <= 256 ? 256 : 512;
-    static_assert(3 * BN + D <= 512, "tensor memory budget");
+    static constexpr int TMEM_Q = 2 * BN + D + BN / 2;
+    static constexpr int TMEM_USED = TMEM_Q + D / 2;
+    static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
+    static_assert(TMEM_USED <= 512, "tensor memory budget");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -153,8 +153,8 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
 
 template <int D, int BN>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const AttnArgs a) {
     using L = Layout<D, BN>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        mbar_init(bars.q_full(), 1);
+        mbar_init(bars.q_full(), 4);  // the softmax warps' elected lanes, once Q is in TMEM
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bars.k_full(s), 1);
             mbar_init(bars.k_empty(s), 1);
@@ -193,7 +193,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_relinquish();
     }
     if (warp == 4 && lane == 0) {
-        prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
     }
@@ -205,12 +204,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == 4) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const int qrow0 = bh * a.Nq + qb * a.T;
             const int krow0 = bh * a.Nk;
-            mbar_arrive_expect_tx(bars.q_full(), L::Q_BYTES);
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-                tma_load_2d(sbase + L::OFF_Q + c * (BM * 128), &tmQ, bars.q_full(), c * 64, qrow0);
             const int32_t* row_idx =
                 a.idx ? a.idx + (static_cast<size_t>(bh) * a.m + qb) * static_cast<size_t>(n)
                       : nullptr;
@@ -249,7 +243,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             // Copies still in flight (only possible after an abort) must land
             // before the CTA exits: wait for the last ones of every slot.
-            drain_wait(bars.q_full(), 0);
             for (int t = issued - 1; t >= 0 && t >= issued - 2 * STAGES; --t) {
                 const int j = t >> 1, s = j % STAGES;
                 const uint32_t par = (j / STAGES) & 1;
@@ -275,12 +268,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const uint32_t d_tmem = tmem + L::TMEM_S + bi * BN;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk & 3) * 32;  // 16 bf16 along K inside a 128-B row
-                    const uint64_t ad =
-                        smem_desc_sw128(sbase + L::OFF_Q + (kk >> 2) * (BM * 128) + off, 16);
+                    // A = Q from tensor memory (8 columns per 16 bf16); B = K_j, whose
+                    // 16-element K slice sits 32 B into its 128-B swizzled row
+                    const uint32_t at = tmem + L::TMEM_Q + kk * 8;
                     const uint64_t bd = smem_desc_sw128(
-                        sbase + L::OFF_K + s * L::KV_TILE + (kk >> 2) * (BN * 128) + off, 16);
-                    mma_bf16_ss(d_tmem, ad, bd, ID_S, kk > 0 ? 1u : 0u);
+                        sbase + L::OFF_K + s * L::KV_TILE + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16);
+                    mma_bf16_ts(d_tmem, at, bd, ID_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bars.k_empty(s));
                 mma_commit(bars.s_full(bi));
@@ -297,7 +290,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     // A = P_j from tensor memory: 16 bf16 of a row = 8 columns
-                    const uint32_t at = tmem + L::TMEM_P + bi * (BN / 2) + kk * 8;
+                    const uint32_t at = tmem + L::TMEM_P + kk * 8;
                     const uint64_t bd = smem_desc_sw128(
                         sbase + L::OFF_V + s * L::KV_TILE + kk * (16 * 128), BN * 128);
                     mma_bf16_ts(tmem + L::TMEM_O, at, bd, ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
@@ -315,6 +308,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float m_run = -INFINITY;
         float l_run = 0.f;
         bool ok = true;
+        {
+            // this thread's query row -> tensor memory as bf16 pairs, the A operand
+            // of every S = Q K^T; rows past the end of Q read as zeros
+            const long long grow =
+                static_cast<long long>(bh) * a.Nq + static_cast<long long>(qb) * a.T + row;
+            float qv[D / 2];
+            if (grow < a.q_rows) {
+                const uint4* src = reinterpret_cast<const uint4*>(a.q + grow * D);
+#pragma unroll
+                for (int u = 0; u < D / 8; ++u) {
+                    const uint4 x = __ldg(src + u);
+                    qv[4 * u + 0] = __uint_as_float(x.x);
+                    qv[4 * u + 1] = __uint_as_float(x.y);
+                    qv[4 * u + 2] = __uint_as_float(x.z);
+                    qv[4 * u + 3] = __uint_as_float(x.w);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < D / 2; ++i) qv[i] = 0.f;
+            }
+            const uint32_t t_q = tmem + lane_base + L::TMEM_Q;
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) tmem_st32(t_q + c * 32, qv + c * 32);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.q_full());
+        }
         for (int j = 0; j < n; ++j) {
             const int bi = j & 1;
             if (!warp_wait(bars.s_full(bi), (j >> 1) & 1, abort_flag)) {
@@ -379,29 +400,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float2 s23 = __fadd2_rn(sum2[2], sum2[3]);
             const float2 s03 = __fadd2_rn(s01, s23);
             const float rs = s03.x + s03.y;
-            // P buffer bi was last read by PV_{j-2}
-            if (j >= 2 && !warp_wait(bars.pv_done(bi), ((j - 2) >> 1) & 1, abort_flag)) {
+            // the P buffer (and O, should it need rescaling) was last read by PV_{j-1}
+            if (j >= 1 && !warp_wait(bars.pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
+            tc_fence_after();
             {
                 // P_j (bf16 pairs, lower key in the low half) into tensor memory
                 float pk[BN / 2];
 #pragma unroll
                 for (int i = 0; i < BN / 2; ++i)
                     pk[i] = __uint_as_float(pack_bf16x2(s[2 * i], s[2 * i + 1]));
-                const uint32_t t_p = tmem + lane_base + L::TMEM_P + bi * (BN / 2);
+                const uint32_t t_p = tmem + lane_base + L::TMEM_P;
 #pragma unroll
                 for (int c = 0; c < BN / 64; ++c) tmem_st32(t_p + c * 32, pk + c * 32);
                 tmem_wait_st();
             }
             if (__any_sync(0xffffffffu, resc)) {
-                // O must hold PV_{j-1} before it is rescaled
-                if (!warp_wait(bars.pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
+                // O holds PV_{j-1} (waited for above) and is rescaled in place
                 const float f = resc ? ex2_approx(m_run - m_new) : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
@@ -492,17 +509,19 @@ template <int D, int BN>
 int launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B,
            cudaStream_t st) {
     using L = Layout<D, BN>;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tk, tv;
     const uint64_t bh = static_cast<uint64_t>(B) * a.H;
-    if (!make_tmap(&tq, q, bh * a.Nq, D, BM) || !make_tmap(&tk, k, bh * a.Nk, D, BN) ||
-        !make_tmap(&tv, v, bh * a.Nk, D, BN))
+    if (!make_tmap(&tk, k, bh * a.Nk, D, BN) || !make_tmap(&tv, v, bh * a.Nk, D, BN))
         return VELOX_ECUDA;
+    AttnArgs args = a;
+    args.q = static_cast<const __nv_bfloat16*>(q);
+    args.q_rows = static_cast<long long>(bh) * a.Nq;
     auto kern = attn_fwd_kernel<D, BN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) !=
         cudaSuccess)
         return VELOX_ECUDA;
     dim3 grid(a.m, a.H, B);
-    kern<<<grid, NTHREADS, L::SMEM, st>>>(tq, tk, tv, a);
+    kern<<<grid, NTHREADS, L::SMEM, st>>>(tk, tv, args);
     return cudaGetLastError() == cudaSuccess ? VELOX_OK : VELOX_ECUDA;
 }
 

@@ -19,6 +19,8 @@ struct AttnArgs {
     __nv_bfloat16* o;
     float* lse;
     int32_t* status;
+    const __nv_bfloat16* q;  // set by the launcher
+    long long q_rows;        // B * H * Nq
 };
 
 int attn_fwd_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B, int d,
