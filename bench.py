@@ -414,6 +414,157 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+def layer_inputs_on_device(torch, case, layers: int, device, seed: int):
+    """Layer 0 is the host-generated case; layers 1.. are drawn on the device
+    with the same structure (Q = N(0,1) + mu_h, past chunk c's K shifted by the
+    chunk's view-overlap proxy times mu_h, V = N(0,1)), one seeded generator per
+    layer. Returns lists of bf16 tensors q[l], k[l], v[l]."""
+    s = case.shape
+    w0 = Workload(case, device)
+    qs, ks, vs = [w0.q], [w0.k], [w0.v]
+    ov = torch.tensor(case.meta["view_overlap"], dtype=torch.float32, device=device)
+    for l in range(1, layers):
+        g = torch.Generator(device=device)
+        g.manual_seed(seed * 1000 + l)
+        mu = 0.5 * torch.randn((s.H, 1, s.d), generator=g, device=device)
+        q = (torch.randn((s.B, s.H, s.Nq, s.d), generator=g, device=device) + mu).to(torch.bfloat16)
+        k = torch.randn((s.B, s.H, s.P + 1, s.Nq, s.d), generator=g, device=device)
+        k[:, :, : s.P] += ov.view(1, 1, s.P, 1, 1) * mu.view(1, s.H, 1, 1, s.d)
+        k = k.view(s.B, s.H, s.Nk, s.d).to(torch.bfloat16)
+        v = torch.randn((s.B, s.H, s.Nk, s.d), generator=g, device=device).to(torch.bfloat16)
+        qs.append(q), ks.append(k), vs.append(v)
+        del k
+    return w0, qs, ks, vs
+
+
+def run_pipeline(args):
+    """One denoising step of the 30-layer pipeline at chunk 48: the geometry
+    (recency-priority multiwarp of the 48 past depth maps -> slices -> overlap
+    counts) runs on a side stream while layer 0 pools its keys; layer 0's
+    selection waits for the counts; then routing + attention for every layer."""
+    import torch
+    from geometry_routed_block_b200 import velox as vx
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    layers = args.layers
+    case = synth.make_case(5, seed=1005 + rank, layers=1)
+    s = case.shape
+    s.layers = layers
+    w, qs, ks, vs = layer_inputs_on_device(torch, case, layers, device, 1005 + rank)
+    peaks, peak_kind = load_peaks()
+
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    past_depth = dev(case.past_depth[0])
+    past_poses, past_intr = dev(case.past_poses[0]), dev(case.past_intr[0])
+    past_cams = dev(np.stack([synth.camera_record(case.past_poses[0, j], case.past_intr[0, j])
+                              for j in range(s.P)]))
+    cur_cam = dev(case.cur_cam)
+    cur_depth = torch.empty((1, s.Hp, s.Wp), dtype=torch.float32, device=device)
+    mw_ws = vx.depth_multiwarp_workspace(s.Hp, s.Wp, device)
+    slices = torch.empty((s.P, 18), dtype=torch.float32, device=device)
+    counts = torch.empty((s.B, s.m, s.P), dtype=torch.int32, device=device)
+    idx = torch.empty((s.B, s.H, s.m, s.topk), dtype=torch.int32, device=device)
+    o = torch.empty_like(qs[0])
+    lse = torch.empty((s.B, s.H, s.Nq), dtype=torch.float32, device=device)
+    ws = w.ws
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream(device=device)
+    ev_start = torch.cuda.Event()
+    ev_geo = torch.cuda.Event()
+
+    def geometry(stream):
+        vx.depth_multiwarp(past_depth, past_cams, cur_cam[0], 0.01, ws=mw_ws, out=cur_depth[0],
+                           stream=stream)
+        vx.slices_build(past_depth, past_poses, past_intr, out=slices, stream=stream)
+        vx.block_overlap(cur_depth, cur_cam, slices[None], s.F, s.T, out=counts, stream=stream)
+
+    def layer(l, ready=None):
+        vx.route_topk(qs[l], ks[l], counts, s.alpha, s.topk, s.T, ws=ws, out=idx, counts_ready=ready)
+        vx.sparse_attn_fwd(qs[l], ks[l], vs[l], idx, s.T, out=o, lse=lse, status=w.status)
+
+    def step_async(ev=None):
+        ev_start.record(main)
+        side.wait_event(ev_start)
+        geometry(side)
+        ev_geo.record(side)
+        if ev is not None:
+            ev[0].record(main)
+            ev[1].record(side)
+        for l in range(layers):
+            layer(l, ev_geo if l == 0 else None)
+            if ev is not None and l == 0:
+                ev[2].record(main)
+        if ev is not None:
+            ev[3].record(main)
+
+    def step_serial():
+        geometry(main)
+        for l in range(layers):
+            layer(l)
+
+    for _ in range(max(3, args.warmup)):
+        step_async()
+    step_serial()
+    torch.cuda.synchronize()
+    steps = max(1, args.steps)
+    # the timed region: K whole steps with the geometry in flight on the side stream
+    with ClockSampler(local) as clk:
+        t_async = time_loop(torch, step_async, steps)
+    clocks = clk.summary()
+    # exposure, per step, from events: when the geometry is done vs when layer 0's
+    # routing (whose selection waited for it) is done; plus the same steps run
+    # serially, interleaved with async ones so clock drift cancels
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    geo_done, route0_done, a_ms, s_ms = [], [], [], []
+    for _ in range(max(2, steps // 2)):
+        ev = [mk() for _ in range(4)]
+        step_async(ev)
+        torch.cuda.synchronize()
+        geo_done.append(ev[0].elapsed_time(ev[1]))
+        route0_done.append(ev[0].elapsed_time(ev[2]))
+        a_ms.append(ev[0].elapsed_time(ev[3]))
+        e0, e1 = mk(), mk()
+        e0.record(main)
+        step_serial()
+        e1.record(main)
+        torch.cuda.synchronize()
+        s_ms.append(e0.elapsed_time(e1))
+    g0, g1 = mk(), mk()
+    torch.cuda.synchronize()
+    g0.record(side)
+    for _ in range(20):
+        geometry(side)
+    g1.record(side)
+    torch.cuda.synchronize()
+    t_geo = g0.elapsed_time(g1) / 20
+    med = statistics.median
+    kf = kept_flops(s) * layers
+    value = world * kf / (t_async * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(t_async, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"denoising step, {layers} layers x " + workload_desc(s)
+                   + "; current depth from the multiwarp of the past depth maps",
+                   "l2": "inputs larger than L2; no flush"},
+        "geometry_ms": round(t_geo, 4),
+        "geometry_done_after_ms": round(med(geo_done), 4),
+        "layer0_routing_done_after_ms": round(med(route0_done), 4),
+        "geometry_exposed_ms": round(max(0.0, med(geo_done) - med(route0_done)), 4),
+        "interleaved_async_step_ms": round(med(a_ms), 4),
+        "interleaved_serial_step_ms": round(med(s_ms), 4),
+        "gpu_launches": (7 + 4 * layers) * steps,
+        "device_status": int(w.status.item()),
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -456,12 +607,15 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
-    ap.add_argument("--workload", default="headline", choices=["headline", "sweep"])
+    ap.add_argument("--workload", default="headline", choices=["headline", "sweep", "pipeline"])
+    ap.add_argument("--layers", type=int, default=30, help="layers (pipeline workload)")
     ap.add_argument("--P", type=int, default=None, help="past chunks (sweep workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "pipeline":
+        run_pipeline(args)
     else:
         run_gpu(args)
 

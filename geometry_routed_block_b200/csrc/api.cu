@@ -59,7 +59,7 @@ size_t velox_route_topk_workspace_size(int B, int H, int Nq, int Nk, int d, int 
 
 int velox_route_topk(const void* q, const void* k, int dtype, int B, int H, int Nq, int Nk, int d,
                      int T, const int32_t* counts, float alpha, int topk, int32_t* idx, void* ws,
-                     size_t ws_bytes, void* stream) {
+                     size_t ws_bytes, void* counts_ready, void* stream) {
     if (!q || !k || !idx || !ws) return VELOX_EINVAL;
     if (dtype != VELOX_BF16 && dtype != VELOX_F32) return VELOX_EUNSUPPORTED;
     if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || d < 1 || T < 1) return VELOX_EINVAL;
@@ -94,6 +94,7 @@ int velox_route_topk(const void* q, const void* k, int dtype, int B, int H, int 
     const size_t qbar_bytes = (rows * d * sizeof(float) + 255) & ~static_cast<size_t>(255);
     r.qbar = static_cast<float*>(ws);
     r.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + qbar_bytes);
+    r.counts_ready = static_cast<cudaEvent_t>(counts_ready);
     return velox::route_launch(q, k, dtype, r, as_stream(stream));
 }
 

@@ -6,10 +6,10 @@
 // CTA owns a 128-row query tile of one (batch, head) and walks only the key
 // blocks listed for its query block.
 //
-// CTA = 6 warps:
+// CTA = 7 warps:
 //   warps 0-3  softmax / correction / epilogue; thread i owns query row i,
 //              which is TMEM lane i
-//   warp 4     TMA producer: K_j and V_j of every listed block
+//   warps 4, 6 TMA producers: K_j (warp 4) and V_j (warp 6) of every listed block
 //              (128-byte swizzled tiles, no multicast)
 //   warp 5     tcgen05 issuer (one thread): S_j = Q K_j^T into a double-buffered
 //              TMEM S; O += P_j V_j. Q and P_j are A operands read from tensor
@@ -38,8 +38,12 @@ namespace velox {
 namespace {
 
 constexpr int BM = 128;          // query rows per CTA tile (MMA M)
-constexpr int NTHREADS = 192;    // 6 warps
-constexpr int STAGES = 3;        // K and V ring depth
+constexpr int NTHREADS = 224;    // 7 warps
+constexpr int KST = 4;           // K ring depth
+constexpr int VST = 3;           // V ring depth
+constexpr int WARP_TMA_K = 4;
+constexpr int WARP_MMA = 5;
+constexpr int WARP_TMA_V = 6;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr float RESCALE_THRESHOLD = 8.0f;          // log2 units
 
@@ -47,10 +51,10 @@ template <int D, int BN>
 struct Layout {
     static constexpr int KV_TILE = BN * D * 2;
     static constexpr int OFF_K = 0;
-    static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
-    static constexpr int OFF_BAR = OFF_V + STAGES * KV_TILE;
+    static constexpr int OFF_V = OFF_K + KST * KV_TILE;
+    static constexpr int OFF_BAR = OFF_V + VST * KV_TILE;
     // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_empty[2], p_full[2], pv_done[2]
-    static constexpr int NBAR = 1 + 4 * STAGES + 8;
+    static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 8;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
@@ -68,14 +72,15 @@ struct Layout {
 struct Bars {
     uint32_t base;
     __device__ uint32_t q_full() const { return base; }
+    static constexpr int R = 1 + 2 * KST + 2 * VST;  // first of the per-block barriers
     __device__ uint32_t k_full(int s) const { return base + 8 * (1 + s); }
-    __device__ uint32_t k_empty(int s) const { return base + 8 * (1 + STAGES + s); }
-    __device__ uint32_t v_full(int s) const { return base + 8 * (1 + 2 * STAGES + s); }
-    __device__ uint32_t v_empty(int s) const { return base + 8 * (1 + 3 * STAGES + s); }
-    __device__ uint32_t s_full(int i) const { return base + 8 * (1 + 4 * STAGES + i); }
-    __device__ uint32_t s_empty(int i) const { return base + 8 * (3 + 4 * STAGES + i); }
-    __device__ uint32_t p_full(int i) const { return base + 8 * (5 + 4 * STAGES + i); }
-    __device__ uint32_t pv_done(int i) const { return base + 8 * (7 + 4 * STAGES + i); }
+    __device__ uint32_t k_empty(int s) const { return base + 8 * (1 + KST + s); }
+    __device__ uint32_t v_full(int s) const { return base + 8 * (1 + 2 * KST + s); }
+    __device__ uint32_t v_empty(int s) const { return base + 8 * (1 + 2 * KST + VST + s); }
+    __device__ uint32_t s_full(int i) const { return base + 8 * (R + i); }
+    __device__ uint32_t s_empty(int i) const { return base + 8 * (R + 2 + i); }
+    __device__ uint32_t p_full(int i) const { return base + 8 * (R + 4 + i); }
+    __device__ uint32_t pv_done(int i) const { return base + 8 * (R + 6 + i); }
 };
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
@@ -174,9 +179,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         mbar_init(bars.q_full(), 4);  // the softmax warps' elected lanes, once Q is in TMEM
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < KST; ++s) {
             mbar_init(bars.k_full(s), 1);
             mbar_init(bars.k_empty(s), 1);
+        }
+        for (int s = 0; s < VST; ++s) {
             mbar_init(bars.v_full(s), 1);
             mbar_init(bars.v_empty(s), 1);
         }
@@ -188,11 +195,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == WARP_MMA) {
         tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == WARP_TMA_K && lane == 0) {
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
     }
@@ -201,9 +208,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
-        // ------------------------------------------------------------ producer
+    if (warp == WARP_TMA_K || warp == WARP_TMA_V) {
+        // ------------------------------------------------------------ producers
+        // one thread streams K_j, another V_j, each into its own ring, so a K
+        // load never queues behind a V slot that is still being read
         if (lane == 0) {
+            const bool is_v = warp == WARP_TMA_V;
+            const int nst = is_v ? VST : KST;
+            const CUtensorMap* tm = is_v ? &tmV : &tmK;
+            const uint32_t ring = sbase + (is_v ? L::OFF_V : L::OFF_K);
+            auto full = [&](int st) { return is_v ? bars.v_full(st) : bars.k_full(st); };
+            auto empty = [&](int st) { return is_v ? bars.v_empty(st) : bars.k_empty(st); };
             const int krow0 = bh * a.Nk;
             const int32_t* row_idx =
                 a.idx ? a.idx + (static_cast<size_t>(bh) * a.m + qb) * static_cast<size_t>(n)
@@ -211,7 +226,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             auto fetch = [&](int j) -> int {
                 int kb = row_idx ? __ldg(row_idx + j) : j;
                 if (kb < 0 || kb >= a.n_kb) {
-                    if (a.status) atomicOr(a.status, VELOX_STATUS_BAD_INDEX);
+                    if (a.status && !is_v) atomicOr(a.status, VELOX_STATUS_BAD_INDEX);
                     kb = 0;
                 }
                 return kb;
@@ -219,37 +234,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int kb = fetch(0);
             int issued = 0;
             for (int j = 0; j < n; ++j) {
-                const int s = j % STAGES;
-                const uint32_t par = ((j / STAGES) - 1) & 1;
+                const int st = j % nst;
                 const int kb_next = (j + 1 < n) ? fetch(j + 1) : 0;
-                const int krow = krow0 + kb * BN;
-                if (j >= STAGES && !mbar_wait(bars.k_empty(s), par, abort_flag, WAIT_LIMIT_NS)) break;
-                mbar_arrive_expect_tx(bars.k_full(s), L::KV_TILE);
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c)
-                    tma_load_2d(sbase + L::OFF_K + s * L::KV_TILE + c * (BN * 128), &tmK,
-                                bars.k_full(s), c * 64, krow);
-                if (j >= STAGES && !mbar_wait(bars.v_empty(s), par, abort_flag, WAIT_LIMIT_NS)) {
-                    issued = 2 * j + 1;
+                if (j >= nst &&
+                    !mbar_wait(empty(st), ((j / nst) - 1) & 1, abort_flag, WAIT_LIMIT_NS))
                     break;
-                }
-                mbar_arrive_expect_tx(bars.v_full(s), L::KV_TILE);
+                mbar_arrive_expect_tx(full(st), L::KV_TILE);
 #pragma unroll
                 for (int c = 0; c < D / 64; ++c)
-                    tma_load_2d(sbase + L::OFF_V + s * L::KV_TILE + c * (BN * 128), &tmV,
-                                bars.v_full(s), c * 64, krow);
-                issued = 2 * j + 2;
+                    tma_load_2d(ring + st * L::KV_TILE + c * (BN * 128), tm, full(st), c * 64,
+                                krow0 + kb * BN);
+                issued = j + 1;
                 kb = kb_next;
             }
             // Copies still in flight (only possible after an abort) must land
-            // before the CTA exits: wait for the last ones of every slot.
-            for (int t = issued - 1; t >= 0 && t >= issued - 2 * STAGES; --t) {
-                const int j = t >> 1, s = j % STAGES;
-                const uint32_t par = (j / STAGES) & 1;
-                drain_wait((t & 1) ? bars.v_full(s) : bars.k_full(s), par);
-            }
+            // before the CTA exits: wait for the last one of every slot.
+            for (int j = issued - 1; j >= 0 && j >= issued - nst; --j)
+                drain_wait(full(j % nst), (j / nst) & 1);
         }
-    } else if (warp == 5) {
+    } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_bf16_f32(BM, BN, false, false);
@@ -257,9 +260,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             bool ok = mbar_wait(bars.q_full(), 0, abort_flag, WAIT_LIMIT_NS);
             tc_fence_after();
             auto issue_s = [&](int j) -> bool {
-                const int s = j % STAGES;
+                const int s = j % KST;
                 const int bi = j & 1;
-                if (!mbar_wait(bars.k_full(s), (j / STAGES) & 1, abort_flag, WAIT_LIMIT_NS))
+                if (!mbar_wait(bars.k_full(s), (j / KST) & 1, abort_flag, WAIT_LIMIT_NS))
                     return false;
                 if (j >= 2 &&
                     !mbar_wait(bars.s_empty(bi), ((j >> 1) - 1) & 1, abort_flag, WAIT_LIMIT_NS))
@@ -282,9 +285,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (ok && n > 0) ok = issue_s(0);
             for (int j = 0; ok && j < n; ++j) {
                 if (j + 1 < n && !issue_s(j + 1)) break;
-                const int s = j % STAGES;
+                const int s = j % VST;
                 const int bi = j & 1;
-                if (!mbar_wait(bars.v_full(s), (j / STAGES) & 1, abort_flag, WAIT_LIMIT_NS)) break;
+                if (!mbar_wait(bars.v_full(s), (j / VST) & 1, abort_flag, WAIT_LIMIT_NS)) break;
                 if (!mbar_wait(bars.p_full(bi), (j >> 1) & 1, abort_flag, WAIT_LIMIT_NS)) break;
                 tc_fence_after();
 #pragma unroll
@@ -470,7 +473,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (threadIdx.x == 0 && *abort_flag && a.status) atomicOr(a.status, VELOX_STATUS_TIMEOUT);
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == WARP_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }

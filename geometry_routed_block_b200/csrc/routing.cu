@@ -9,14 +9,15 @@
 // Kernels:
 //   pool_q      qbar[b,h,qb,:] = mean of the T query rows of block qb (fp32)
 //   pool_score  streams the past keys once (16-byte loads): pools each key
-//               block, dots it with every qbar of its head and writes the
-//               modulated score s' = qbar.kbar / sqrt(d) (+ alpha * count / T
-//               on covered query blocks). Eight consecutive key blocks form
-//               one work item so each query block's scores leave as one
-//               32-byte sector.
-//   select      one warp per (b, h, qb): radix select of the (topk - m)
-//               largest s' over the past blocks (equal s': smaller index
-//               first), then the m current-chunk blocks; ascending indices.
+//               block and dots it with every qbar of its head, writing the
+//               block importance s = qbar.kbar / sqrt(d). One warp pools one
+//               key block at a time; warps run independently.
+//   select      one warp per (b, h, qb): applies the modulation
+//               s' = s + alpha * count / T on covered query blocks, then
+//               selects exactly the (topk - m) largest s' over the past blocks (equal s': smaller index
+//               first) by bitwise bisection on order-preserving keys held in
+//               registers (radix select beyond 4096 blocks), then the m
+//               current-chunk blocks; ascending indices.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -29,7 +30,6 @@ namespace velox {
 namespace {
 
 constexpr int POOL_THREADS = 256;
-constexpr int KGROUP = 8;  // key blocks per pool_score work item
 
 template <typename TIn>
 struct VecTraits;
@@ -105,64 +105,113 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_q_kernel(const TIn* __restr
     if (threadIdx.x < D) qbar[blk * D + threadIdx.x] = out[threadIdx.x];
 }
 
+// One warp pools one [T][D] block: lane (cg, r0) reads 16-byte column group cg
+// of rows r0, r0 + RPW, ... (all its loads in flight at once, in batches),
+// sums in fp32 pairs, then the lanes of a column group reduce by shuffles.
+// On return every lane holds the column sums of its group, times 1/T.
+template <typename TIn, int D, int T>
+__device__ __forceinline__ void warp_pool(const TIn* __restrict__ blk, int lane, float* kbar) {
+    using V = VecTraits<TIn>;
+    constexpr int TPR = D / V::VEC;
+    constexpr int RPW = 32 / TPR;
+    constexpr int LOADS = T / RPW;
+    constexpr int BATCH = LOADS < 16 ? LOADS : 16;
+    const int cg = lane % TPR, r0 = lane / TPR;
+    const TIn* base = blk + static_cast<size_t>(r0) * D + cg * V::VEC;
+    float acc[V::VEC];
+#pragma unroll
+    for (int i = 0; i < V::VEC; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int b0 = 0; b0 < LOADS; b0 += BATCH) {
+        uint4 buf[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i)
+            buf[i] = ldg_stream(base + static_cast<size_t>(b0 + i) * RPW * D);
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) V::add(acc, buf[i]);
+    }
+#pragma unroll
+    for (int o = TPR; o < 32; o <<= 1) {
+#pragma unroll
+        for (int i = 0; i < V::VEC; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    }
+#pragma unroll
+    for (int i = 0; i < V::VEC; ++i) kbar[i] = acc[i] * (1.0f / T);
+}
+
+// CTA = one (b, h) slice of the grid; each warp walks its own past key blocks
+// (kb = blockIdx.x * WARPS + warp, strided by the grid), pools one block at a
+// time and scores it against every query block of its head straight from
+// shared memory. Warps never wait for one another after the q-bar load.
 template <typename TIn, int D, int T>
 __global__ void __launch_bounds__(POOL_THREADS)
     pool_score_kernel(const TIn* __restrict__ k, const float* __restrict__ qbar, RouteArgs r) {
     using V = VecTraits<TIn>;
+    constexpr int TPR = D / V::VEC;
+    constexpr int RPW = 32 / TPR;
+    constexpr int WARPS = POOL_THREADS / 32;
     extern __shared__ float dsm[];
-    float* q_s = dsm;                                  // [m][D]
-    float* kb_s = q_s + r.m * D;                       // [KGROUP][D]
-    float* red = kb_s + KGROUP * D;                    // [RPP][D]
-    int* cov_s = reinterpret_cast<int*>(red + (POOL_THREADS / (D / V::VEC)) * D);  // [m]
+    float* q_s = dsm;  // [m][D]
 
     const int bh = blockIdx.y;
-    const int b = bh / r.H;
     const int t = threadIdx.x;
     for (int i = t; i < r.m * D; i += POOL_THREADS) q_s[i] = qbar[static_cast<size_t>(bh) * r.m * D + i];
-    const int32_t* cnt = r.counts ? r.counts + static_cast<size_t>(b) * r.m * r.P : nullptr;
-    for (int qb = t; qb < r.m; qb += POOL_THREADS) {
-        int any = 0;
-        if (cnt)
-            for (int j = 0; j < r.P; ++j) any |= (cnt[qb * r.P + j] > 0);
-        cov_s[qb] = any;
-    }
     __syncthreads();
 
     const TIn* kh = k + static_cast<size_t>(bh) * r.Nk * D;
-    const int n_groups = (r.n_past + KGROUP - 1) / KGROUP;
     const int warp = t >> 5, lane = t & 31;
-    const float invT = 1.0f / T;
-    for (int g = blockIdx.x; g < n_groups; g += gridDim.x) {
-        const int kb0 = g * KGROUP;
-        const int nk = min(KGROUP, r.n_past - kb0);
-        for (int i = 0; i < nk; ++i)
-            pool_block<TIn, D, T>(kh + static_cast<size_t>(kb0 + i) * T * D, kb_s + i * D, red);
-        // scores: warp w takes query blocks w, w+8, ...; lanes split d
-        for (int qb = warp; qb < r.m; qb += POOL_THREADS / 32) {
-            float qv[D / 32];
+    const int cg = lane % TPR, r0 = lane / TPR;
+    float* srow = r.scores + static_cast<size_t>(bh) * r.m * r.n_past;
+    for (int kb = blockIdx.x * WARPS + warp; kb < r.n_past; kb += gridDim.x * WARPS) {
+        float kv[V::VEC];
+        warp_pool<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, kv);
+        // every lane runs the same number of iterations (full-warp shuffles)
+        for (int q0 = 0; q0 < r.m; q0 += RPW) {
+            const int qb = q0 + r0;
+            const bool valid = qb < r.m;
+            float p = 0.f;
+            if (valid) {
+                const float* qrow = q_s + qb * D + cg * V::VEC;
 #pragma unroll
-            for (int u = 0; u < D / 32; ++u) qv[u] = q_s[qb * D + lane + 32 * u];
-            float mine = 0.f;
-#pragma unroll
-            for (int i = 0; i < KGROUP; ++i) {
-                float p = 0.f;
-                if (i < nk) {
-#pragma unroll
-                    for (int u = 0; u < D / 32; ++u) p = fmaf(qv[u], kb_s[i * D + lane + 32 * u], p);
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-                if (lane == i) mine = p;
+                for (int i = 0; i < V::VEC; ++i) p = fmaf(qrow[i], kv[i], p);
             }
-            if (lane < nk) {
-                const int kb = kb0 + lane;
-                float s = mine * r.inv_sqrt_d;
-                if (cov_s[qb]) s = s + r.alpha * static_cast<float>(cnt[qb * r.P + kb / r.m]) * invT;
-                r.scores[(static_cast<size_t>(bh) * r.m + qb) * r.n_past + kb] = s;
-            }
+#pragma unroll
+            for (int o = 1; o < TPR; o <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+            if (valid && cg == 0) srow[static_cast<size_t>(qb) * r.n_past + kb] = p * r.inv_sqrt_d;
         }
-        __syncthreads();
     }
+}
+
+struct SelArgs {
+    const float* scores;  // [rows][n_past] raw block scores
+    int rows, n_past, m, H, P, k_past, topk;
+    const int32_t* counts;  // [B][m][P] or nullptr
+    float alpha, invT;
+    int32_t* idx;
+};
+
+// Geometric modulation of one row: s' = s + alpha * count[chunk(kb)] / T when
+// the query block is covered (some count > 0), s' = s otherwise.
+struct RowMod {
+    const int32_t* cnt;  // counts[b][qb][*] or nullptr when uncovered / no geometry
+    float alpha, invT;
+    int m;
+    __device__ __forceinline__ float operator()(float sc, int kb) const {
+        return cnt ? sc + alpha * static_cast<float>(cnt[kb / m]) * invT : sc;
+    }
+};
+
+__device__ __forceinline__ RowMod row_mod(const SelArgs& a, int row) {
+    RowMod r{nullptr, a.alpha, a.invT, a.m};
+    if (a.counts) {
+        const int qb = row % a.m;
+        const int b = (row / a.m) / a.H;
+        const int32_t* c = a.counts + (static_cast<size_t>(b) * a.m + qb) * a.P;
+        int any = 0;
+        for (int j = 0; j < a.P; ++j) any |= (c[j] > 0);
+        if (any) r.cnt = c;
+    }
+    return r;
 }
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -171,16 +220,17 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 constexpr int SEL_WARPS = 8;
+constexpr int SEL_REG_WARPS = 4;
 
-__global__ void __launch_bounds__(SEL_WARPS * 32)
-    select_kernel(const float* __restrict__ scores, int rows, int n_past, int m, int k_past, int topk,
-                  int32_t* __restrict__ idx) {
+__global__ void __launch_bounds__(SEL_WARPS * 32) select_kernel(const SelArgs a) {
     __shared__ uint32_t hist_all[SEL_WARPS][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * SEL_WARPS + warp;
-    if (row >= rows) return;
-    const float* sc = scores + static_cast<size_t>(row) * n_past;
-    int32_t* out = idx + static_cast<size_t>(row) * topk;
+    if (row >= a.rows) return;
+    const int n_past = a.n_past, m = a.m, k_past = a.k_past;
+    const float* sc = a.scores + static_cast<size_t>(row) * n_past;
+    int32_t* out = a.idx + static_cast<size_t>(row) * a.topk;
+    const RowMod mod = row_mod(a, row);
     for (int i = lane; i < m; i += 32) out[k_past + i] = n_past + i;
     if (k_past <= 0) return;
     if (k_past >= n_past) {
@@ -196,7 +246,7 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
         for (int i = lane; i < 256; i += 32) h[i] = 0;
         __syncwarp();
         for (int i = lane; i < n_past; i += 32) {
-            const uint32_t key = order_key(sc[i]);
+            const uint32_t key = order_key(mod(sc[i], i));
             if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
         }
         __syncwarp();
@@ -242,7 +292,7 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
     int written = 0, eq_seen = 0;
     for (int base = 0; base < n_past; base += 32) {
         const int i = base + lane;
-        const uint32_t key = i < n_past ? order_key(sc[i]) : 0u;
+        const uint32_t key = i < n_past ? order_key(mod(sc[i], i)) : 0u;
         const bool gt = i < n_past && key > prefix;
         const bool eq = i < n_past && key == prefix;
         const unsigned eqb = __ballot_sync(FULL, eq);
@@ -254,15 +304,92 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
     }
 }
 
+// Register-resident selection for rows of at most 32 * CH past blocks: lane l
+// keeps the keys of blocks l, l + 32, ... ; the (k_past)-th largest key is found
+// bit by bit from the top (largest u with count(key >= u) >= k_past: 32
+// rounds of compares and a warp popcount), then a ballot pass emits every
+// larger key and the first equal ones in index order. Padding keys are 0,
+// below every real key.
+template <int CH>
+__global__ void __launch_bounds__(SEL_REG_WARPS * 32)
+    select_reg_kernel(const SelArgs a) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * SEL_REG_WARPS + warp;
+    if (row >= a.rows) return;
+    const int n_past = a.n_past, m = a.m, k_past = a.k_past;
+    const float* sc = a.scores + static_cast<size_t>(row) * n_past;
+    int32_t* out = a.idx + static_cast<size_t>(row) * a.topk;
+    const RowMod mod = row_mod(a, row);
+    for (int i = lane; i < m; i += 32) out[k_past + i] = n_past + i;
+    if (k_past <= 0) return;
+    if (k_past >= n_past) {
+        for (int i = lane; i < n_past; i += 32) out[i] = i;
+        return;
+    }
+    const unsigned FULL = 0xffffffffu;
+    uint32_t key[CH];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        const int i = c * 32 + lane;
+        key[c] = i < n_past ? order_key(mod(__ldg(sc + i), i)) : 0u;
+    }
+    uint32_t u = 0;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = u | (1u << bit);
+        int c4[4] = {0, 0, 0, 0};  // independent partial counts
+#pragma unroll
+        for (int c = 0; c < CH; ++c) c4[c & 3] += key[c] >= cand ? 1 : 0;
+        int cnt = (c4[0] + c4[1]) + (c4[2] + c4[3]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o);
+        if (cnt >= k_past) u = cand;
+    }
+    int gt = 0;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) gt += key[c] > u ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(FULL, gt, o);
+    const int remaining = k_past - gt;
+    const unsigned lt = (1u << lane) - 1u;
+    int written = 0, eq_seen = 0;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        const int i = c * 32 + lane;
+        const bool eq = i < n_past && key[c] == u;
+        const unsigned eqb = __ballot_sync(FULL, eq);
+        const bool take = (key[c] > u) || (eq && (eq_seen + __popc(eqb & lt)) < remaining);
+        const unsigned tb = __ballot_sync(FULL, take);
+        if (take) out[written + __popc(tb & lt)] = i;
+        written += __popc(tb);
+        eq_seen += __popc(eqb);
+    }
+}
+
+int select_launch(const SelArgs& a, cudaStream_t st) {
+    const dim3 grid((a.rows + SEL_REG_WARPS - 1) / SEL_REG_WARPS), block(SEL_REG_WARPS * 32);
+    if (a.n_past <= 32 * 2)
+        select_reg_kernel<2><<<grid, block, 0, st>>>(a);
+    else if (a.n_past <= 32 * 8)
+        select_reg_kernel<8><<<grid, block, 0, st>>>(a);
+    else if (a.n_past <= 32 * 32)
+        select_reg_kernel<32><<<grid, block, 0, st>>>(a);
+    else if (a.n_past <= 32 * 64)
+        select_reg_kernel<64><<<grid, block, 0, st>>>(a);
+    else if (a.n_past <= 32 * 128)
+        select_reg_kernel<128><<<grid, block, 0, st>>>(a);
+    else
+        select_kernel<<<(a.rows + SEL_WARPS - 1) / SEL_WARPS, SEL_WARPS * 32, 0, st>>>(a);
+    return VELOX_OK;
+}
+
 template <typename TIn, int D, int T>
 int route_typed(const TIn* q, const TIn* k, const RouteArgs& r, cudaStream_t st) {
     using V = VecTraits<TIn>;
     const int BH = r.B * r.H;
     pool_q_kernel<TIn, D, T><<<BH * r.m, POOL_THREADS, 0, st>>>(q, r.qbar);
     if (r.n_past > 0) {
-        const size_t smem = (static_cast<size_t>(r.m) * D + KGROUP * D +
-                             (POOL_THREADS / (D / V::VEC)) * D) * sizeof(float) +
-                            static_cast<size_t>(r.m) * sizeof(int);
+        const size_t smem = static_cast<size_t>(r.m) * D * sizeof(float);
         auto kern = pool_score_kernel<TIn, D, T>;
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -271,15 +398,18 @@ int route_typed(const TIn* q, const TIn* k, const RouteArgs& r, cudaStream_t st)
         int dev = 0, sms = 148;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int n_groups = (r.n_past + KGROUP - 1) / KGROUP;
-        // about 4 resident CTAs per SM over all heads
+        // about 4 resident CTAs per SM over all heads, never more warps than blocks
+        const int warps = POOL_THREADS / 32;
         int gx = (4 * sms + BH - 1) / BH;
-        gx = max(1, min(gx, n_groups));
+        gx = max(1, min(gx, (r.n_past + warps - 1) / warps));
         pool_score_kernel<TIn, D, T><<<dim3(gx, BH), POOL_THREADS, smem, st>>>(k, r.qbar, r);
     }
-    const int rows = BH * r.m;
-    select_kernel<<<(rows + SEL_WARPS - 1) / SEL_WARPS, SEL_WARPS * 32, 0, st>>>(
-        r.scores, rows, r.n_past, r.m, r.topk - r.m, r.topk, r.idx);
+    // the counts are read by the selection only: it may wait for them alone
+    if (r.counts_ready && cudaStreamWaitEvent(st, r.counts_ready, 0) != cudaSuccess)
+        return VELOX_ECUDA;
+    SelArgs sa{r.scores, BH * r.m, r.n_past, r.m, r.H, r.P, r.topk - r.m, r.topk,
+               r.counts, r.alpha, 1.0f / static_cast<float>(T), r.idx};
+    select_launch(sa, st);
     return cudaGetLastError() == cudaSuccess ? VELOX_OK : VELOX_ECUDA;
 }
 

@@ -41,6 +41,7 @@ struct RouteArgs {
     int32_t* idx;
     float* qbar;    // workspace [B*H*m][d]
     float* scores;  // workspace [B*H*m][n_past]
+    cudaEvent_t counts_ready;  // selection waits for it when set
 };
 size_t route_ws_bytes(int B, int H, int m, int n_past, int d);
 int route_launch(const void* q, const void* k, int dtype, const RouteArgs& r, cudaStream_t st);

@@ -42,7 +42,7 @@ SIGNATURES = {
                                      _vp, _vp]),
     "velox_route_topk_workspace_size": (_c_size, [_c_int] * 6),
     "velox_route_topk": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
-                                  _vp, _c_float, _c_int, _vp, _vp, _c_size, _vp]),
+                                  _vp, _c_float, _c_int, _vp, _vp, _c_size, _vp, _vp]),
     "velox_sparse_attn_fwd": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                        _c_int, _c_int, _c_float, _vp, _vp, _vp, _vp]),
     "velox_depth_multiwarp_workspace_size": (_c_size, [_c_int, _c_int]),
@@ -165,9 +165,11 @@ def route_workspace(B: int, H: int, Nq: int, Nk: int, d: int, T: int, device="cu
 
 def route_topk(q: torch.Tensor, k: torch.Tensor, counts: torch.Tensor | None, alpha: float,
                topk: int, T: int, ws: torch.Tensor | None = None, out: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
+               counts_ready: torch.cuda.Event | None = None, stream=None) -> torch.Tensor:
     """q [B,H,Nq,d], k [B,H,Nk,d] (bf16 or f32), counts [B,m,P] int32 or None ->
-    idx [B,H,m,topk] int32 (ascending key-block indices)."""
+    idx [B,H,m,topk] int32 (ascending key-block indices). With `counts_ready`,
+    only the selection kernel waits for that event (the counts' producer may
+    still be running on another stream while the keys are pooled)."""
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
     if q.dtype != k.dtype:
@@ -181,8 +183,9 @@ def route_topk(q: torch.Tensor, k: torch.Tensor, counts: torch.Tensor | None, al
         ws = route_workspace(B, H, Nq, Nk, d, T, q.device)
     if out is None:
         out = torch.empty((B, H, Nq // T, topk), dtype=torch.int32, device=q.device)
+    ev = ctypes.c_void_p(counts_ready.cuda_event) if counts_ready is not None else None
     _check(lib.velox_route_topk(_ptr(q), _ptr(k), dtype, B, H, Nq, Nk, d, T, _ptr(counts),
-                                float(alpha), int(topk), _ptr(out), _ptr(ws), ws.numel(),
+                                float(alpha), int(topk), _ptr(out), _ptr(ws), ws.numel(), ev,
                                 _stream(stream)), "velox_route_topk")
     return out
 

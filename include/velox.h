@@ -133,6 +133,10 @@ VELOX_API size_t velox_route_topk_workspace_size(int B, int H, int Nq, int Nk, i
  *   counts [B][m][P] int32 from velox_block_overlap, or NULL (no geometry)
  *   idx    [B][H][m][topk] int32 output: selected key blocks, ascending
  *   ws     scratch of velox_route_topk_workspace_size bytes (256-B aligned)
+ *   counts_ready  a cudaEvent_t or NULL. When set, only the final selection
+ *          kernel waits for it (cudaStreamWaitEvent): pooling and scoring, which
+ *          do not read the counts, run meanwhile -- so the geometry (slices,
+ *          overlap) can be produced on another stream at the same time.
  * with m = Nq/T query blocks, P = Nk/Nq - 1 past chunks, n_past = P*m past key
  * blocks, and key block kb covering keys [kb*T, (kb+1)*T).
  * Readings implemented:
@@ -149,7 +153,7 @@ VELOX_API size_t velox_route_topk_workspace_size(int B, int H, int Nq, int Nk, i
  */
 VELOX_API int velox_route_topk(const void* q, const void* k, int dtype, int B, int H, int Nq, int Nk, int d,
                      int T, const int32_t* counts, float alpha, int topk, int32_t* idx, void* ws,
-                     size_t ws_bytes, void* stream);
+                     size_t ws_bytes, void* counts_ready, void* stream);
 
 /*
  * Block-sparse attention forward over the routed blocks (step 4 of

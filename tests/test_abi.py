@@ -56,12 +56,13 @@ NULL = None
 def test_route_topk_rejects(lib):
     f = lib.velox_route_topk
     ok = dict(q=FAKE, k=FAKE, dtype=0, B=1, H=2, Nq=256, Nk=1280, d=64, T=64, counts=NULL,
-              alpha=2.0, topk=6, idx=FAKE, ws=FAKE, ws_bytes=1 << 30, stream=NULL)
+              alpha=2.0, topk=6, idx=FAKE, ws=FAKE, ws_bytes=1 << 30, ready=NULL, stream=NULL)
 
     def call(**kw):
         a = {**ok, **kw}
         return f(a["q"], a["k"], a["dtype"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"], a["T"],
-                 a["counts"], a["alpha"], a["topk"], a["idx"], a["ws"], a["ws_bytes"], a["stream"])
+                 a["counts"], a["alpha"], a["topk"], a["idx"], a["ws"], a["ws_bytes"], a["ready"],
+                 a["stream"])
 
     assert call(q=NULL) == -1
     assert call(idx=NULL) == -1

@@ -286,3 +286,59 @@ def test_rollout_p96_routing_sampled_heads(vx):
     idx = vx.route_topk(dev(c.q[0]), dev(c.k[0]), dev(counts), s.alpha, s.topk, s.T)
     want, s_mod = vo.route_topk(c.q[0], c.k[0], counts, s.alpha, s.topk, s.T)
     assert compare_selection(idx.cpu().numpy(), want, s_mod, s.m) <= 3
+
+
+def test_route_exact_ties_break_to_the_smaller_index(vx):
+    # past chunks 0-2 are copies, and so are 3-5: their pooled scores tie exactly
+    # (in fp32 on the device and in fp64 in the oracle), so the selection is
+    # fixed by the tie-break alone
+    rng = np.random.default_rng(21)
+    T, d, B, H, m = 64, 64, 1, 2, 2
+    Nq = m * T
+    q = rng.standard_normal((B, H, Nq, d), dtype=np.float32)
+    base = rng.standard_normal((2, B, H, Nq, d), dtype=np.float32)
+    cur = rng.standard_normal((B, H, Nq, d), dtype=np.float32)
+    k = np.concatenate([base[0]] * 3 + [base[1]] * 3 + [cur], axis=2)
+    for dtype in ("f32", "bf16"):
+        qq, kk = (q, k) if dtype == "f32" else (synth.f32_to_bf16_bits(q), synth.f32_to_bf16_bits(k))
+        for topk in (m + 1, m + 2, m + 5, m + 7, m + 11):
+            got = vx.route_topk(dev(qq), dev(kk), None, 0.0, topk, T).cpu().numpy()
+            want, _ = vo.route_topk(qq, kk, None, 0.0, topk, T)
+            assert np.array_equal(got, want), (dtype, topk)
+
+
+def test_pipeline_async_geometry_matches_serial_and_oracle(vx):
+    """Multiwarp -> slices -> overlap on a side stream while the keys are
+    pooled; the selection waits for the counts through an event. Same result as
+    running everything on one stream, and as the oracle (sampled heads)."""
+    c = synth.make_case(5, layers=1)
+    s = c.shape
+    cams = np.stack([synth.camera_record(c.past_poses[0, j], c.past_intr[0, j]) for j in range(s.P)])
+    q, k = dev(c.q[0]), dev(c.k[0])
+    pd, poses, intr = dev(c.past_depth[0]), dev(c.past_poses[0]), dev(c.past_intr[0])
+    cur = dev(c.cur_cam)
+
+    def geometry(stream=None):
+        depth = vx.depth_multiwarp(pd, dev(cams), cur[0], 0.01, stream=stream)
+        sl = vx.slices_build(pd, poses, intr, stream=stream)
+        return vx.block_overlap(depth[None], cur, sl[None], s.F, s.T, stream=stream)
+
+    serial_counts = geometry()
+    serial = vx.route_topk(q, k, serial_counts, s.alpha, s.topk, s.T)
+    side = torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+    ev0, ev = torch.cuda.Event(), torch.cuda.Event()
+    ev0.record(main)
+    side.wait_event(ev0)
+    async_counts = geometry(stream=side)
+    ev.record(side)
+    async_idx = vx.route_topk(q, k, async_counts, s.alpha, s.topk, s.T, counts_ready=ev)
+    torch.cuda.synchronize()
+    assert torch.equal(serial_counts, async_counts) and torch.equal(serial, async_idx)
+    depth = vo.depth_multiwarp(c.past_depth[0], cams, c.cur_cam[0], 0.01)
+    sl = vo.slices_build(c.past_depth[0], c.past_poses[0], c.past_intr[0])
+    counts = vo.block_overlap(depth[None], c.cur_cam, sl[None], s.F, s.T)
+    assert np.array_equal(async_counts.cpu().numpy(), counts)
+    heads = [2, 17]
+    want, s_mod = vo.route_topk(c.q[0][:, heads], c.k[0][:, heads], counts, s.alpha, s.topk, s.T)
+    assert compare_selection(async_idx[:, heads].cpu().numpy(), want, s_mod, s.m) <= 2
