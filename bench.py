@@ -481,22 +481,23 @@ def run_pipeline(args):
         vx.slices_build(past_depth, past_poses, past_intr, out=slices, stream=stream)
         vx.block_overlap(cur_depth, cur_cam, slices[None], s.F, s.T, out=counts, stream=stream)
 
-    def layer(l, ready=None):
+    def layer(l, ready=None, routed=None):
         vx.route_topk(qs[l], ks[l], counts, s.alpha, s.topk, s.T, ws=ws, out=idx, counts_ready=ready)
+        if routed is not None:
+            routed.record(main)
         vx.sparse_attn_fwd(qs[l], ks[l], vs[l], idx, s.T, out=o, lse=lse, status=w.status)
 
     def step_async(ev=None):
         ev_start.record(main)
+        if ev is not None:
+            ev[0].record(main)  # origin, before any geometry is enqueued
         side.wait_event(ev_start)
         geometry(side)
         ev_geo.record(side)
         if ev is not None:
-            ev[0].record(main)
-            ev[1].record(side)
+            ev[1].record(side)  # geometry done
         for l in range(layers):
-            layer(l, ev_geo if l == 0 else None)
-            if ev is not None and l == 0:
-                ev[2].record(main)
+            layer(l, ev_geo if l == 0 else None, ev[2] if (ev is not None and l == 0) else None)
         if ev is not None:
             ev[3].record(main)
 

@@ -53,16 +53,16 @@ struct Layout {
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + KST * KV_TILE;
     static constexpr int OFF_BAR = OFF_V + VST * KV_TILE;
-    // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_empty[2], p_full[2], pv_done[2]
-    static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 8;
+    // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2], pv_done[2]
+    static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
-    // tensor memory columns: S[2] (fp32), O (fp32), P (bf16 pairs), Q (bf16 pairs)
+    // tensor memory columns: S[2] (fp32; P_j, as bf16 pairs, overwrites the
+    // first BN/2 columns of S_j once S_j has been read), O (fp32), Q (bf16 pairs)
     static constexpr int TMEM_S = 0;
     static constexpr int TMEM_O = 2 * BN;
-    static constexpr int TMEM_P = 2 * BN + D;
-    static constexpr int TMEM_Q = 2 * BN + D + BN / 2;
+    static constexpr int TMEM_Q = 2 * BN + D;
     static constexpr int TMEM_USED = TMEM_Q + D / 2;
     static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
     static_assert(TMEM_USED <= 512, "tensor memory budget");
@@ -78,9 +78,8 @@ struct Bars {
     __device__ uint32_t v_full(int s) const { return base + 8 * (1 + 2 * KST + s); }
     __device__ uint32_t v_empty(int s) const { return base + 8 * (1 + 2 * KST + VST + s); }
     __device__ uint32_t s_full(int i) const { return base + 8 * (R + i); }
-    __device__ uint32_t s_empty(int i) const { return base + 8 * (R + 2 + i); }
-    __device__ uint32_t p_full(int i) const { return base + 8 * (R + 4 + i); }
-    __device__ uint32_t pv_done(int i) const { return base + 8 * (R + 6 + i); }
+    __device__ uint32_t p_full(int i) const { return base + 8 * (R + 2 + i); }
+    __device__ uint32_t pv_done(int i) const { return base + 8 * (R + 4 + i); }
 };
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
@@ -189,8 +188,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bars.s_full(i), 1);
-            mbar_init(bars.s_empty(i), 4);  // one elected arrive per softmax warp
-            mbar_init(bars.p_full(i), 4);
+            mbar_init(bars.p_full(i), 4);  // one elected arrive per softmax warp
             mbar_init(bars.pv_done(i), 1);
         }
         fence_mbar_init();
@@ -264,9 +262,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int bi = j & 1;
                 if (!mbar_wait(bars.k_full(s), (j / KST) & 1, abort_flag, WAIT_LIMIT_NS))
                     return false;
-                if (j >= 2 &&
-                    !mbar_wait(bars.s_empty(bi), ((j >> 1) - 1) & 1, abort_flag, WAIT_LIMIT_NS))
-                    return false;
+                // S buffer bi last held P_{j-2}, read by PV_{j-2}, which this
+                // thread issued earlier: MMAs from one thread run in issue order
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + L::TMEM_S + bi * BN;
 #pragma unroll
@@ -293,7 +290,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     // A = P_j from tensor memory: 16 bf16 of a row = 8 columns
-                    const uint32_t at = tmem + L::TMEM_P + kk * 8;
+                    const uint32_t at = tmem + L::TMEM_S + bi * BN + kk * 8;
                     const uint64_t bd = smem_desc_sw128(
                         sbase + L::OFF_V + s * L::KV_TILE + kk * (16 * 128), BN * 128);
                     mma_bf16_ts(tmem + L::TMEM_O, at, bd, ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
@@ -365,9 +362,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int c = HALF / 32; c < BN / 32; ++c) reg_fence32(s + c * 32);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bars.s_empty(bi));  // S buffer may be overwritten
             max_range<HALF, BN>(s, acc);
             float mx = max3f(max3f(acc[0], acc[1], acc[2]), max3f(acc[3], acc[4], acc[5]),
                              fmaxf(acc[6], acc[7]));
@@ -403,25 +397,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float2 s23 = __fadd2_rn(sum2[2], sum2[3]);
             const float2 s03 = __fadd2_rn(s01, s23);
             const float rs = s03.x + s03.y;
-            // the P buffer (and O, should it need rescaling) was last read by PV_{j-1}
-            if (j >= 1 && !warp_wait(bars.pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
             {
                 // P_j (bf16 pairs, lower key in the low half) into tensor memory
                 float pk[BN / 2];
 #pragma unroll
                 for (int i = 0; i < BN / 2; ++i)
                     pk[i] = __uint_as_float(pack_bf16x2(s[2 * i], s[2 * i + 1]));
-                const uint32_t t_p = tmem + lane_base + L::TMEM_P;
+                // into the S buffer just read: PV_j reads it from there
+                const uint32_t t_p = tmem + lane_base + L::TMEM_S + bi * BN;
 #pragma unroll
                 for (int c = 0; c < BN / 64; ++c) tmem_st32(t_p + c * 32, pk + c * 32);
                 tmem_wait_st();
             }
             if (__any_sync(0xffffffffu, resc)) {
-                // O holds PV_{j-1} (waited for above) and is rescaled in place
+                // O must hold PV_{j-1} before it is rescaled in place
+                if (!warp_wait(bars.pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
                 const float f = resc ? ex2_approx(m_run - m_new) : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
