@@ -42,6 +42,26 @@ METRIC = "chunk-48 routed attention ms & TFLOP/s (kept blocks), speedup vs dense
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes of one sparse attention launch at this workload, from the ncu capture
+# summarised in profiles/attn_pp_kernel_chunk48_dram.md; reported only while the
+# kernel sources still hash to what was captured.
+ATTN_TRAFFIC = {
+    "bytes_per_launch": 642.25e6 + 22.86e6,
+    "sources": {"attention_pp.cu": "c5c73d0285dee029", "attn_common.cuh": "edbf6bcdb3a2cde6",
+                "ptx.cuh": "34475d094993081f"},
+}
+
+
+def attn_traffic():
+    import hashlib
+    base = os.path.join(ROOT, "geometry_routed_block_b200", "csrc")
+    for name, want in ATTN_TRAFFIC["sources"].items():
+        with open(os.path.join(base, name), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != want:
+                return None
+    return ATTN_TRAFFIC["bytes_per_launch"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -374,13 +394,14 @@ def run_gpu(args):
         "allowed_speedup": round(s.nKB / s.topk, 3),
         "roofline": {
             "bound": "tensor",
-            "kernel": "attn_fwd_kernel<128,128> (sparse, kept blocks)",
+            "kernel": "attn_pp_kernel (sparse walk, kept blocks)",
             "achieved": round(attn_tflops, 2),
             "peak": peak_t,
             "peak_kind": f"bf16 sustained ({peak_kind})",
             "unit": "TFLOP/s",
             "frac": round(attn_tflops / peak_t, 4),
-            "traffic": None,
+            "frac_of_burst": round(attn_tflops / peaks["bf16_tflops"], 4),
+            "traffic": attn_traffic() if s.P == 48 and cfg == 3 else None,
         },
         "routing_roofline": {
             "bound": "hbm", "achieved": round(route_gbs, 1), "peak": peaks["hbm_gbs"],

@@ -74,6 +74,7 @@ int velox_route_topk(const void* q, const void* k, int dtype, int B, int H, int 
     const size_t need = velox_route_topk_workspace_size(B, H, Nq, Nk, d, T);
     if (need == 0 || ws_bytes < need) return VELOX_EINVAL;
     if (static_cast<long long>(B) * H * Nk * d >= (1ll << 40)) return VELOX_EINVAL;
+    if (Nk / T > 8192) return VELOX_EINVAL;  // key-block index range of the selection
 
     velox::RouteArgs r{};
     r.B = B;

@@ -30,8 +30,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "ptx.cuh"
-#include "velox_internal.cuh"
+#include "attn_common.cuh"
 
 namespace velox {
 
@@ -44,8 +43,6 @@ constexpr int VST = 3;           // V ring depth
 constexpr int WARP_TMA_K = 4;
 constexpr int WARP_MMA = 5;
 constexpr int WARP_TMA_V = 6;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any legitimate wait
-constexpr float RESCALE_THRESHOLD = 8.0f;          // log2 units
 
 template <int D, int BN>
 struct Layout {
@@ -81,79 +78,6 @@ struct Bars {
     __device__ uint32_t p_full(int i) const { return base + 8 * (R + 2 + i); }
     __device__ uint32_t pv_done(int i) const { return base + 8 * (R + 4 + i); }
 };
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-                 "r"(d)
-                 : "memory");
-}
-
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-// acc[k] = max(acc[k], s[LO + k + 8 i]) over [LO, HI): 8 independent chains,
-// three-input max where possible
-template <int LO, int HI>
-__device__ __forceinline__ void max_range(const float* s, float* acc) {
-    int i = LO;
-#pragma unroll
-    for (; i + 16 <= HI; i += 16) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = max3f(acc[k], s[i + k], s[i + 8 + k]);
-    }
-#pragma unroll
-    for (; i + 8 <= HI; i += 8) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = fmaxf(acc[k], s[i + k]);
-    }
-}
-
-// 2^x for two lanes on the FMA pipe (Cody-Waite range reduction + minimax
-// cubic; coefficients from geometry_routed_block_b200/exp2_poly.py, relative
-// error < 1e-4). n = round(x) comes from the low mantissa bits of
-// x + 1.5 * 2^23; f = x - n lies in [-1/2, 1/2]; the result is p(f) with n added
-// to its exponent field. x is clamped to [-120, inf): below that 2^x is
-// negligible next to the row sum, and the exponent cannot wrap.
-constexpr float EXP2_C0 = 0.9999280571937561f;
-constexpr float EXP2_C1 = 0.6932609677314758f;
-constexpr float EXP2_C2 = 0.2426111251115799f;
-constexpr float EXP2_C3 = 0.0551716685295105f;
-constexpr unsigned EXP2_EMU_MASK = 0x52;  // pairs 1, 4 and 6 of every 8
-
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    x.x = fmaxf(x.x, -120.f);
-    x.y = fmaxf(x.y, -120.f);
-    const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
-    const float2 t = __fadd2_rn(x, magic);
-    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-    float2 p = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
-    p = __ffma2_rn(p, f, make_float2(EXP2_C1, EXP2_C1));
-    p = __ffma2_rn(p, f, make_float2(EXP2_C0, EXP2_C0));
-    float2 r;
-    r.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
-    r.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
-    return r;
-}
-
-// bounded wait, made uniform across the warp (a warp leaves together)
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-    bool ok = mbar_wait(bar, parity, abort, WAIT_LIMIT_NS);
-    return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
-    // waits for copies already in flight; ignores the abort flag, short limit
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > 100000000ull) return false;
-    }
-    return true;
-}
 
 template <int D, int BN>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -473,7 +397,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+template <int D, int BN>
+int launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B,
+           cudaStream_t st) {
+    using L = Layout<D, BN>;
+    CUtensorMap tk, tv;
+    const uint64_t bh = static_cast<uint64_t>(B) * a.H;
+    if (!make_tmap(&tk, k, bh * a.Nk, D, BN) || !make_tmap(&tv, v, bh * a.Nk, D, BN))
+        return VELOX_ECUDA;
+    AttnArgs args = a;
+    args.q = static_cast<const __nv_bfloat16*>(q);
+    args.q_rows = static_cast<long long>(bh) * a.Nq;
+    auto kern = attn_fwd_kernel<D, BN>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) !=
+        cudaSuccess)
+        return VELOX_ECUDA;
+    dim3 grid(a.m, a.H, B);
+    kern<<<grid, NTHREADS, L::SMEM, st>>>(tk, tv, args);
+    return cudaGetLastError() == cudaSuccess ? VELOX_OK : VELOX_ECUDA;
+}
+
+}  // namespace
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag flag;
     std::call_once(flag, [] {
@@ -502,31 +448,9 @@ bool make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols,
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN>
-int launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B,
-           cudaStream_t st) {
-    using L = Layout<D, BN>;
-    CUtensorMap tk, tv;
-    const uint64_t bh = static_cast<uint64_t>(B) * a.H;
-    if (!make_tmap(&tk, k, bh * a.Nk, D, BN) || !make_tmap(&tv, v, bh * a.Nk, D, BN))
-        return VELOX_ECUDA;
-    AttnArgs args = a;
-    args.q = static_cast<const __nv_bfloat16*>(q);
-    args.q_rows = static_cast<long long>(bh) * a.Nq;
-    auto kern = attn_fwd_kernel<D, BN>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) !=
-        cudaSuccess)
-        return VELOX_ECUDA;
-    dim3 grid(a.m, a.H, B);
-    kern<<<grid, NTHREADS, L::SMEM, st>>>(tk, tv, args);
-    return cudaGetLastError() == cudaSuccess ? VELOX_OK : VELOX_ECUDA;
-}
-
-}  // namespace
-
 int attn_fwd_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B, int d,
                     cudaStream_t st) {
-    if (d == 128 && a.T == 128) return launch<128, 128>(q, k, v, a, B, st);
+    if (d == 128 && a.T == 128) return attn_pp_launch(q, k, v, a, B, st);
     if (d == 128 && a.T == 64) return launch<128, 64>(q, k, v, a, B, st);
     if (d == 64 && a.T == 128) return launch<64, 128>(q, k, v, a, B, st);
     if (d == 64 && a.T == 64) return launch<64, 64>(q, k, v, a, B, st);

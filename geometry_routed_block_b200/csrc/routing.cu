@@ -195,21 +195,28 @@ struct SelArgs {
 struct RowMod {
     const int32_t* cnt;  // counts[b][qb][*] or nullptr when uncovered / no geometry
     float alpha, invT;
-    int m;
+    float inv_m;
+    // chunk(kb) = kb / m as floor((kb + 1/2) / m): the quotient sits at least
+    // 1/(2m) from an integer and the product is accurate to ~1e-4 for
+    // kb < 2^13, so the conversion truncates to the exact integer quotient
     __device__ __forceinline__ float operator()(float sc, int kb) const {
-        return cnt ? sc + alpha * static_cast<float>(cnt[kb / m]) * invT : sc;
+        if (!cnt) return sc;
+        const int chunk = __float2int_rz(__fmul_rn(static_cast<float>(kb) + 0.5f, inv_m));
+        return sc + alpha * static_cast<float>(__ldg(cnt + chunk)) * invT;
     }
 };
 
-__device__ __forceinline__ RowMod row_mod(const SelArgs& a, int row) {
-    RowMod r{nullptr, a.alpha, a.invT, a.m};
+// Called by all 32 lanes of a warp: the lanes read the row's counts in
+// parallel and a ballot decides whether the query block is covered.
+__device__ __forceinline__ RowMod row_mod(const SelArgs& a, int row, int lane) {
+    RowMod r{nullptr, a.alpha, a.invT, 1.0f / static_cast<float>(a.m)};
     if (a.counts) {
         const int qb = row % a.m;
         const int b = (row / a.m) / a.H;
         const int32_t* c = a.counts + (static_cast<size_t>(b) * a.m + qb) * a.P;
-        int any = 0;
-        for (int j = 0; j < a.P; ++j) any |= (c[j] > 0);
-        if (any) r.cnt = c;
+        bool any = false;
+        for (int j = lane; j < a.P; j += 32) any |= __ldg(c + j) > 0;
+        if (__any_sync(0xffffffffu, any)) r.cnt = c;
     }
     return r;
 }
@@ -230,7 +237,7 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_kernel(const SelArgs a)
     const int n_past = a.n_past, m = a.m, k_past = a.k_past;
     const float* sc = a.scores + static_cast<size_t>(row) * n_past;
     int32_t* out = a.idx + static_cast<size_t>(row) * a.topk;
-    const RowMod mod = row_mod(a, row);
+    const RowMod mod = row_mod(a, row, lane);
     for (int i = lane; i < m; i += 32) out[k_past + i] = n_past + i;
     if (k_past <= 0) return;
     if (k_past >= n_past) {
@@ -319,7 +326,7 @@ __global__ void __launch_bounds__(SEL_REG_WARPS * 32)
     const int n_past = a.n_past, m = a.m, k_past = a.k_past;
     const float* sc = a.scores + static_cast<size_t>(row) * n_past;
     int32_t* out = a.idx + static_cast<size_t>(row) * a.topk;
-    const RowMod mod = row_mod(a, row);
+    const RowMod mod = row_mod(a, row, lane);
     for (int i = lane; i < m; i += 32) out[k_past + i] = n_past + i;
     if (k_past <= 0) return;
     if (k_past >= n_past) {

@@ -10,7 +10,7 @@ import numpy as np
 from geometry_routed_block_b200 import exp2_poly
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                   "geometry_routed_block_b200", "csrc", "attention.cu")
+                   "geometry_routed_block_b200", "csrc", "attn_common.cuh")
 
 
 def kernel_constants():
