@@ -132,6 +132,73 @@ int velox_sparse_attn_fwd(const void* q, const void* k, const void* v, const int
     return velox::attn_fwd_launch(q, k, v, a, B, d, as_stream(stream));
 }
 
+size_t velox_kbar_cache_bytes(int B, int H, int max_past_chunks, int Nq, int d, int T) {
+    if (B < 1 || H < 1 || max_past_chunks < 1 || T < 1 || Nq < T || Nq % T || d < 1) return 0;
+    return static_cast<size_t>(B) * H * max_past_chunks * (Nq / T) * d * sizeof(float);
+}
+
+int velox_kbar_append(const void* k, int dtype, int B, int H, int Nk, int Nq, int d, int T, int chunk,
+                      float* kbar, int max_past_chunks, void* stream) {
+    if (!k || !kbar) return VELOX_EINVAL;
+    if (dtype != VELOX_BF16 && dtype != VELOX_F32) return VELOX_EUNSUPPORTED;
+    if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || d < 1 || T < 1 || max_past_chunks < 1)
+        return VELOX_EINVAL;
+    if (!tile_ok(T) || !tile_ok(d)) return VELOX_EUNSUPPORTED;
+    if (Nq % T || Nk % T) return VELOX_EINVAL;
+    if (chunk < 0 || chunk >= max_past_chunks || static_cast<long long>(chunk + 1) * Nq > Nk)
+        return VELOX_EINVAL;
+    if (!aligned(k, 16) || !aligned(kbar, 16)) return VELOX_EINVAL;
+    if (static_cast<long long>(B) * H > 65535) return VELOX_EINVAL;
+    return velox::kbar_append_launch(k, dtype, B * H, Nk, Nq, d, T, chunk, max_past_chunks * (Nq / T),
+                                     kbar, as_stream(stream));
+}
+
+int velox_route_topk_cached(const void* q, int dtype, const float* kbar, int max_past_chunks, int B,
+                            int H, int Nq, int P, int d, int T, const int32_t* counts, float alpha,
+                            int topk, int32_t* idx, void* ws, size_t ws_bytes, void* counts_ready,
+                            void* stream) {
+    if (!q || !idx || !ws || (P > 0 && !kbar)) return VELOX_EINVAL;
+    if (dtype != VELOX_BF16 && dtype != VELOX_F32) return VELOX_EUNSUPPORTED;
+    if (B < 1 || H < 1 || Nq < 1 || d < 1 || T < 1 || P < 0 || P > max_past_chunks)
+        return VELOX_EINVAL;
+    if (!tile_ok(T) || !tile_ok(d)) return VELOX_EUNSUPPORTED;
+    if (Nq % T) return VELOX_EINVAL;
+    if (!aligned(q, 16) || !aligned(ws, 256) || !aligned(idx, 4) || (kbar && !aligned(kbar, 16)))
+        return VELOX_EINVAL;
+    if (!std::isfinite(alpha)) return VELOX_EINVAL;
+    const long long Nk = static_cast<long long>(P + 1) * Nq;
+    if (Nk >= (1ll << 31) || Nk / T > 8192) return VELOX_EINVAL;
+    const int m = Nq / T;
+    const int n_kb = static_cast<int>(Nk / T);
+    if (topk < m || topk > n_kb) return VELOX_EINVAL;
+    const size_t need = velox_route_topk_workspace_size(B, H, Nq, static_cast<int>(Nk), d, T);
+    if (need == 0 || ws_bytes < need) return VELOX_EINVAL;
+
+    velox::RouteArgs r{};
+    r.B = B;
+    r.H = H;
+    r.Nq = Nq;
+    r.Nk = static_cast<int>(Nk);
+    r.d = d;
+    r.T = T;
+    r.m = m;
+    r.P = P;
+    r.n_past = P * m;
+    r.topk = topk;
+    r.counts = P > 0 ? counts : nullptr;
+    r.alpha = alpha;
+    r.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+    r.idx = idx;
+    const size_t rows = static_cast<size_t>(B) * H * m;
+    const size_t qbar_bytes = (rows * d * sizeof(float) + 255) & ~static_cast<size_t>(255);
+    r.qbar = static_cast<float*>(ws);
+    r.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + qbar_bytes);
+    r.counts_ready = static_cast<cudaEvent_t>(counts_ready);
+    r.kbar = kbar;
+    r.kbar_cap = max_past_chunks * m;
+    return velox::route_launch(q, nullptr, dtype, r, as_stream(stream));
+}
+
 size_t velox_depth_multiwarp_workspace_size(int Hp, int Wp) {
     if (Hp < 1 || Wp < 1) return 0;
     return velox::multiwarp_ws_bytes(Hp * Wp);

@@ -143,7 +143,10 @@ __device__ __forceinline__ void warp_pool(const TIn* __restrict__ blk, int lane,
 // (kb = blockIdx.x * WARPS + warp, strided by the grid), pools one block at a
 // time and scores it against every query block of its head straight from
 // shared memory. Warps never wait for one another after the q-bar load.
-template <typename TIn, int D, int T>
+// CACHED: the pooled key blocks come from a k-bar cache filled by
+// kbar_append_kernel (same pooling code, so the values are bit-identical)
+// instead of being pooled from K here.
+template <typename TIn, int D, int T, bool CACHED>
 __global__ void __launch_bounds__(POOL_THREADS)
     pool_score_kernel(const TIn* __restrict__ k, const float* __restrict__ qbar, RouteArgs r) {
     using V = VecTraits<TIn>;
@@ -164,7 +167,20 @@ __global__ void __launch_bounds__(POOL_THREADS)
     float* srow = r.scores + static_cast<size_t>(bh) * r.m * r.n_past;
     for (int kb = blockIdx.x * WARPS + warp; kb < r.n_past; kb += gridDim.x * WARPS) {
         float kv[V::VEC];
-        warp_pool<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, kv);
+        if constexpr (CACHED) {
+            const float4* src = reinterpret_cast<const float4*>(
+                r.kbar + (static_cast<size_t>(bh) * r.kbar_cap + kb) * D + cg * V::VEC);
+#pragma unroll
+            for (int i = 0; i < V::VEC / 4; ++i) {
+                const float4 x = __ldg(src + i);
+                kv[4 * i + 0] = x.x;
+                kv[4 * i + 1] = x.y;
+                kv[4 * i + 2] = x.z;
+                kv[4 * i + 3] = x.w;
+            }
+        } else {
+            warp_pool<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, kv);
+        }
         // every lane runs the same number of iterations (full-warp shuffles)
         for (int q0 = 0; q0 < r.m; q0 += RPW) {
             const int qb = q0 + r0;
@@ -179,6 +195,33 @@ __global__ void __launch_bounds__(POOL_THREADS)
             for (int o = 1; o < TPR; o <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
             if (valid && cg == 0) srow[static_cast<size_t>(qb) * r.n_past + kb] = p * r.inv_sqrt_d;
         }
+    }
+}
+
+// Pools the m key blocks of one chunk of every (b, h) into the k-bar cache:
+// kbar[bh][chunk * m + i][:] = mean of K rows [chunk * Nq + i * T, + T).
+template <typename TIn, int D, int T>
+__global__ void __launch_bounds__(POOL_THREADS)
+    kbar_append_kernel(const TIn* __restrict__ k, int Nk, int Nq, int m, int chunk, int cap,
+                       float* __restrict__ kbar) {
+    using V = VecTraits<TIn>;
+    constexpr int TPR = D / V::VEC;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = blockIdx.x * (POOL_THREADS / 32) + warp;
+    if (i >= m) return;
+    const int bh = blockIdx.y;
+    const int cg = lane % TPR, r0 = lane / TPR;
+    float kv[V::VEC];
+    warp_pool<TIn, D, T>(k + (static_cast<size_t>(bh) * Nk + static_cast<size_t>(chunk) * Nq +
+                              static_cast<size_t>(i) * T) * D,
+                         lane, kv);
+    if (r0 == 0) {
+        float4* dst = reinterpret_cast<float4*>(
+            kbar + (static_cast<size_t>(bh) * cap + static_cast<size_t>(chunk) * m + i) * D +
+            cg * V::VEC);
+#pragma unroll
+        for (int j = 0; j < V::VEC / 4; ++j)
+            dst[j] = make_float4(kv[4 * j], kv[4 * j + 1], kv[4 * j + 2], kv[4 * j + 3]);
     }
 }
 
@@ -397,7 +440,7 @@ int route_typed(const TIn* q, const TIn* k, const RouteArgs& r, cudaStream_t st)
     pool_q_kernel<TIn, D, T><<<BH * r.m, POOL_THREADS, 0, st>>>(q, r.qbar);
     if (r.n_past > 0) {
         const size_t smem = static_cast<size_t>(r.m) * D * sizeof(float);
-        auto kern = pool_score_kernel<TIn, D, T>;
+        auto kern = r.kbar ? pool_score_kernel<TIn, D, T, true> : pool_score_kernel<TIn, D, T, false>;
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
@@ -409,7 +452,7 @@ int route_typed(const TIn* q, const TIn* k, const RouteArgs& r, cudaStream_t st)
         const int warps = POOL_THREADS / 32;
         int gx = (4 * sms + BH - 1) / BH;
         gx = max(1, min(gx, (r.n_past + warps - 1) / warps));
-        pool_score_kernel<TIn, D, T><<<dim3(gx, BH), POOL_THREADS, smem, st>>>(k, r.qbar, r);
+        kern<<<dim3(gx, BH), POOL_THREADS, smem, st>>>(k, r.qbar, r);
     }
     // the counts are read by the selection only: it may wait for them alone
     if (r.counts_ready && cudaStreamWaitEvent(st, r.counts_ready, 0) != cudaSuccess)
@@ -431,7 +474,36 @@ int route_dispatch(const void* q, const void* k, const RouteArgs& r, cudaStream_
     return VELOX_EUNSUPPORTED;
 }
 
+template <typename TIn, int D, int T>
+int append_typed(const TIn* k, int BH, int Nk, int Nq, int chunk, int cap, float* kbar,
+                 cudaStream_t st) {
+    const int m = Nq / T;
+    const int warps = POOL_THREADS / 32;
+    kbar_append_kernel<TIn, D, T><<<dim3((m + warps - 1) / warps, BH), POOL_THREADS, 0, st>>>(
+        k, Nk, Nq, m, chunk, cap, kbar);
+    return cudaGetLastError() == cudaSuccess ? VELOX_OK : VELOX_ECUDA;
+}
+
+template <typename TIn>
+int append_dispatch(const void* k, int BH, int Nk, int Nq, int d, int T, int chunk, int cap,
+                    float* kbar, cudaStream_t st) {
+    const TIn* tk = static_cast<const TIn*>(k);
+    if (d == 128 && T == 128) return append_typed<TIn, 128, 128>(tk, BH, Nk, Nq, chunk, cap, kbar, st);
+    if (d == 128 && T == 64) return append_typed<TIn, 128, 64>(tk, BH, Nk, Nq, chunk, cap, kbar, st);
+    if (d == 64 && T == 128) return append_typed<TIn, 64, 128>(tk, BH, Nk, Nq, chunk, cap, kbar, st);
+    if (d == 64 && T == 64) return append_typed<TIn, 64, 64>(tk, BH, Nk, Nq, chunk, cap, kbar, st);
+    return VELOX_EUNSUPPORTED;
+}
+
 }  // namespace
+
+int kbar_append_launch(const void* k, int dtype, int BH, int Nk, int Nq, int d, int T, int chunk,
+                       int cap, float* kbar, cudaStream_t st) {
+    if (dtype == VELOX_BF16)
+        return append_dispatch<__nv_bfloat16>(k, BH, Nk, Nq, d, T, chunk, cap, kbar, st);
+    if (dtype == VELOX_F32) return append_dispatch<float>(k, BH, Nk, Nq, d, T, chunk, cap, kbar, st);
+    return VELOX_EUNSUPPORTED;
+}
 
 size_t route_ws_bytes(int B, int H, int m, int n_past, int d) {
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };

@@ -42,9 +42,14 @@ struct RouteArgs {
     float* qbar;    // workspace [B*H*m][d]
     float* scores;  // workspace [B*H*m][n_past]
     cudaEvent_t counts_ready;  // selection waits for it when set
+    const float* kbar;         // k-bar cache [B*H][kbar_cap][d], or nullptr: pool K here
+    int kbar_cap;              // blocks per (b, h) in the cache
 };
 size_t route_ws_bytes(int B, int H, int m, int n_past, int d);
 int route_launch(const void* q, const void* k, int dtype, const RouteArgs& r, cudaStream_t st);
+
+int kbar_append_launch(const void* k, int dtype, int BH, int Nk, int Nq, int d, int T, int chunk,
+                       int cap, float* kbar, cudaStream_t st);
 
 int cast_bf16_launch(const float* x, uint16_t* y, size_t n, cudaStream_t st);
 

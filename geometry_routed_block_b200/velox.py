@@ -51,6 +51,12 @@ SIGNATURES = {
     "velox_cast_bf16": (_c_int, [_vp, _vp, _c_size, _vp]),
     "velox_depth_multiwarp_noalloc": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_float,
                                                _vp, _vp]),
+    "velox_kbar_cache_bytes": (_c_size, [_c_int] * 6),
+    "velox_kbar_append": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                   _vp, _c_int, _vp]),
+    "velox_route_topk_cached": (_c_int, [_vp, _c_int, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                         _c_int, _c_int, _vp, _c_float, _c_int, _vp, _vp, _c_size,
+                                         _vp, _vp]),
 }
 
 
@@ -187,6 +193,55 @@ def route_topk(q: torch.Tensor, k: torch.Tensor, counts: torch.Tensor | None, al
     _check(lib.velox_route_topk(_ptr(q), _ptr(k), dtype, B, H, Nq, Nk, d, T, _ptr(counts),
                                 float(alpha), int(topk), _ptr(out), _ptr(ws), ws.numel(), ev,
                                 _stream(stream)), "velox_route_topk")
+    return out
+
+
+# ---------------------------------------------------------------- pooled-key cache
+
+def kbar_cache(B: int, H: int, max_past_chunks: int, Nq: int, d: int, T: int,
+               device="cuda") -> torch.Tensor:
+    """An empty pooled-key cache [B, H, max_past_chunks * Nq/T, d] float32."""
+    if lib.velox_kbar_cache_bytes(B, H, max_past_chunks, Nq, d, T) == 0:
+        raise VeloxError("velox_kbar_cache_bytes", VELOX_EINVAL)
+    return torch.empty((B, H, max_past_chunks * (Nq // T), d), dtype=torch.float32, device=device)
+
+
+def kbar_append(k: torch.Tensor, Nq: int, T: int, chunk: int, kbar: torch.Tensor,
+                stream=None) -> torch.Tensor:
+    """Pools chunk `chunk` of the KV cache k [B,H,Nk,d] into kbar."""
+    B, H, Nk, d = k.shape
+    dtype = {torch.bfloat16: VELOX_BF16, torch.float32: VELOX_F32}.get(k.dtype)
+    if dtype is None:
+        raise TypeError(f"unsupported dtype {k.dtype}")
+    _expect(kbar, torch.float32, "kbar")
+    max_chunks = kbar.shape[2] // (Nq // T)
+    _check(lib.velox_kbar_append(_ptr(k), dtype, B, H, Nk, Nq, d, T, int(chunk), _ptr(kbar),
+                                 max_chunks, _stream(stream)), "velox_kbar_append")
+    return kbar
+
+
+def route_topk_cached(q: torch.Tensor, kbar: torch.Tensor, P: int, counts: torch.Tensor | None,
+                      alpha: float, topk: int, T: int, ws: torch.Tensor | None = None,
+                      out: torch.Tensor | None = None, counts_ready: torch.cuda.Event | None = None,
+                      stream=None) -> torch.Tensor:
+    """route_topk over P past chunks whose pooled keys are in kbar."""
+    B, H, Nq, d = q.shape
+    dtype = {torch.bfloat16: VELOX_BF16, torch.float32: VELOX_F32}.get(q.dtype)
+    if dtype is None:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    _expect(kbar, torch.float32, "kbar")
+    if counts is not None:
+        _expect(counts, torch.int32, "counts")
+    max_chunks = kbar.shape[2] // (Nq // T)
+    if ws is None:
+        ws = route_workspace(B, H, Nq, (P + 1) * Nq, d, T, q.device)
+    if out is None:
+        out = torch.empty((B, H, Nq // T, topk), dtype=torch.int32, device=q.device)
+    ev = ctypes.c_void_p(counts_ready.cuda_event) if counts_ready is not None else None
+    _check(lib.velox_route_topk_cached(_ptr(q), dtype, _ptr(kbar), max_chunks, B, H, Nq, int(P), d,
+                                       T, _ptr(counts), float(alpha), int(topk), _ptr(out),
+                                       _ptr(ws), ws.numel(), ev, _stream(stream)),
+           "velox_route_topk_cached")
     return out
 
 

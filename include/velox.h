@@ -178,6 +178,40 @@ VELOX_API int velox_sparse_attn_fwd(const void* q, const void* k, const void* v,
                           int topk, int B, int H, int Nq, int Nk, int d, int T, float scale,
                           void* o, float* lse, int32_t* status, void* stream);
 
+/*
+ * Pooled-key cache (an incremental form of the routing's key pooling; the
+ * block importance the model computes in each layer, "Tiefenanalyse" step 3,
+ * only ever needs the mean of each past key block, and a past chunk's keys
+ * never change once the chunk is done).
+ * The cache holds, per (b, h), the mean of each T-token key block of up to
+ * max_past_chunks chunks: kbar [B][H][max_past_chunks * m][d] float32, m = Nq/T.
+ */
+VELOX_API size_t velox_kbar_cache_bytes(int B, int H, int max_past_chunks, int Nq, int d, int T);
+
+/*
+ * Pools the m key blocks of chunk `chunk` (keys [chunk*Nq, (chunk+1)*Nq) of every
+ * (b, h) of the KV cache k [B][H][Nk][d], dtype VELOX_BF16 or VELOX_F32) into
+ * kbar[b][h][chunk*m + i][:]. Call it once per chunk, when the chunk is done.
+ * The values are bit-identical to the pooling velox_route_topk does itself.
+ * Errors: VELOX_EINVAL for sizes that are not multiples, chunk outside
+ * [0, max_past_chunks), keys [chunk*Nq, (chunk+1)*Nq) beyond Nk, NULL or
+ * misaligned (16 B) pointers; VELOX_EUNSUPPORTED as velox_route_topk.
+ */
+VELOX_API int velox_kbar_append(const void* k, int dtype, int B, int H, int Nk, int Nq, int d, int T,
+                                int chunk, float* kbar, int max_past_chunks, void* stream);
+
+/*
+ * velox_route_topk with the past key blocks taken from the pooled-key cache
+ * instead of K: P past chunks (P <= max_past_chunks, chunks 0..P-1 appended)
+ * and the current chunk, Nk = (P + 1) * Nq. Same arguments, semantics,
+ * workspace (velox_route_topk_workspace_size(B, H, Nq, (P+1)*Nq, d, T)) and
+ * errors; the selected blocks equal velox_route_topk's on the same keys.
+ */
+VELOX_API int velox_route_topk_cached(const void* q, int dtype, const float* kbar,
+                                      int max_past_chunks, int B, int H, int Nq, int P, int d, int T,
+                                      const int32_t* counts, float alpha, int topk, int32_t* idx,
+                                      void* ws, size_t ws_bytes, void* counts_ready, void* stream);
+
 /* Bytes of scratch velox_depth_multiwarp needs (0 on bad sizes). */
 VELOX_API size_t velox_depth_multiwarp_workspace_size(int Hp, int Wp);
 

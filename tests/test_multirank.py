@@ -1,0 +1,54 @@
+"""The multi-GPU host logic of bench.py on CPU: two gloo ranks (127.0.0.1).
+Each rank times its own chunk; the job time is the max over ranks and the
+whole-job rate counts every rank's work (weak scaling, no data collective)."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import torch.distributed as dist
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    import bench
+    ms = [3.0 + rank, 10.0 - 4 * rank]           # rank 0: (3, 10), rank 1: (4, 6)
+    got = bench.reduce_max(ms)
+    value = bench.job_throughput(world, 2.0e12, got[0])
+    out[rank] = (got, value, bench.rank_seed(3, rank))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_max_and_count_every_rank():
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    for rank in range(world):
+        got, value, seed = res[rank]
+        assert got == [4.0, 10.0]
+        assert value == pytest.approx(world * 2.0e12 / 4.0e-3)
+        assert seed == 1003 + rank
+    assert res[0][2] != res[1][2]  # the ranks run different chunks
+
+
+def test_single_process_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.reduce_max([1.5, 2.5]) == [1.5, 2.5]
+    assert bench.job_throughput(1, 1e12, 1.0) == pytest.approx(1e15)

@@ -342,3 +342,40 @@ def test_pipeline_async_geometry_matches_serial_and_oracle(vx):
     heads = [2, 17]
     want, s_mod = vo.route_topk(c.q[0][:, heads], c.k[0][:, heads], counts, s.alpha, s.topk, s.T)
     assert compare_selection(async_idx[:, heads].cpu().numpy(), want, s_mod, s.m) <= 2
+
+
+# ---------------------------------------------------------------- pooled-key cache
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_kbar_cache_matches_oracle_pooling(vx, cfg):
+    c = synth.make_case(cfg)
+    s = c.shape
+    k = dev(c.k[0])
+    kbar = vx.kbar_cache(s.B, s.H, s.P, s.Nq, s.d, s.T)
+    for j in range(s.P):
+        vx.kbar_append(k, s.Nq, s.T, j, kbar)
+    want = vo.pool_blocks(c.k[0][:, :, : s.P * s.Nq], s.T)
+    got = kbar.cpu().numpy().astype(np.float64)
+    assert np.abs(got - want).max() <= 1e-6 * max(1.0, np.abs(want).max())
+
+
+@pytest.mark.parametrize("cfg", [1, 3])
+def test_cached_routing_equals_streaming_routing(vx, cfg):
+    c = synth.make_case(cfg)
+    s = c.shape
+    q, k = dev(c.q[0]), dev(c.k[0])
+    if cfg == 1:
+        counts = vx.block_overlap(dev(c.cur_depth), dev(c.cur_cam), dev(c.past_cams), s.F, s.T)
+    else:
+        sl = vx.slices_build(dev(c.past_depth[0]), dev(c.past_poses[0]), dev(c.past_intr[0]))
+        counts = vx.block_overlap(dev(c.cur_depth), dev(c.cur_cam), sl[None], s.F, s.T)
+    kbar = vx.kbar_cache(s.B, s.H, s.P + 3, s.Nq, s.d, s.T)  # spare capacity
+    for j in range(s.P):
+        vx.kbar_append(k, s.Nq, s.T, j, kbar)
+    for alpha in (0.0, s.alpha):
+        want = vx.route_topk(q, k, counts, alpha, s.topk, s.T)
+        got = vx.route_topk_cached(q, kbar, s.P, counts, alpha, s.topk, s.T)
+        assert torch.equal(got, want)
+    # no past chunk yet: only the current chunk's blocks
+    only = vx.route_topk_cached(q, kbar, 0, None, s.alpha, s.m, s.T).cpu().numpy()
+    assert (only == np.arange(s.m)).all()
