@@ -46,8 +46,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # summarised in profiles/attn_pp_kernel_chunk48_dram.md; reported only while the
 # kernel sources still hash to what was captured.
 ATTN_TRAFFIC = {
-    "bytes_per_launch": 642.25e6 + 22.86e6,
-    "sources": {"attention_pp.cu": "c5c73d0285dee029", "attn_common.cuh": "edbf6bcdb3a2cde6",
+    "bytes_per_launch": 642.18e6 + 22.82e6,
+    "sources": {"attention_pp.cu": "13e4340e74204946", "attn_common.cuh": "edbf6bcdb3a2cde6",
                 "ptx.cuh": "34475d094993081f"},
 }
 

@@ -18,10 +18,11 @@
 //   warps 0-3   softmax / correction / epilogue of block A (row = TMEM lane)
 //   warps 4-7   the same for block B
 //   warp 8      TMA producer of the K tiles, in consumption order A0 B0 A1 B1 ...
+//               (2-deep ring: one slot per block)
 //   warp 9      tcgen05 issuer (one thread)
 //   warp 10     TMA producer of the V tiles, same order
 //   warp 11     idle
-// Shared memory: Q_A, Q_B (32 KB each), K ring (3 x 32 KB), V ring (2 x 32 KB),
+// Shared memory: Q_A, Q_B (32 KB each), K ring (2 x 32 KB), V ring (2 x 32 KB),
 // all 128-byte swizzled. Tensor memory (512 columns): S_A, S_B (128 fp32
 // columns each; P, as bf16 pairs, overwrites the upper half of S once S has
 // been read), O_A, O_B (128 fp32 columns each).
@@ -38,11 +39,16 @@ namespace {
 constexpr int PP_THREADS = 384;
 constexpr int PP_D = 128;
 constexpr int PP_BN = 128;
-constexpr int PP_KST = 3;
+constexpr int PP_KST = 2;
 constexpr int PP_VST = 2;
 constexpr int PP_WARP_TMA_K = 8;
 constexpr int PP_WARP_MMA = 9;
 constexpr int PP_WARP_TMA_V = 10;
+// Every exponential goes to the ex2 unit here: with two blocks in flight the
+// softmax has slack, and moving part of the exponentials to the FMA pipe
+// (as the single-block kernel does) only adds issue pressure (measured on the
+// chunk-48 walk: 0/8 of the pairs emulated 1,171 TFLOP/s, 3/8 1,152, 4/8 1,091).
+constexpr unsigned PP_EMU_MASK = 0x00;
 
 struct PPLayout {
     static constexpr int TILE = 128 * 128 * 2;  // a Q, K or V tile: 128 rows x 128 bf16
@@ -81,7 +87,7 @@ __device__ __forceinline__ void exp_half(float* s, float sl2, float m, float2* s
 #pragma unroll
     for (int i = 0; i < 64; i += 2) {
         float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), sc2, ng2);
-        if ((EXP2_EMU_MASK >> ((i >> 1) & 7)) & 1) {
+        if ((PP_EMU_MASK >> ((i >> 1) & 7)) & 1) {
             x = exp2_poly2(x);
         } else {
             x.x = ex2_approx(x.x);
@@ -192,8 +198,23 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                 const int st = l % nst;
                 const int nl = l + 1;
                 const int kb_next = nl < total ? fetch(nl % ntile, nl / ntile) : 0;
-                if (l >= nst && !mbar_wait(empty(st), ((l / nst) - 1) & 1, abort_flag, WAIT_LIMIT_NS))
-                    break;
+                if (l >= nst) {
+                    // With two blocks each ring holds one tile per block, so a slot
+                    // is free once that block's previous S (or P V) is complete:
+                    // wait on that completion barrier (it cannot run two phases
+                    // ahead: the block's next GEMM needs the tile loaded here). A
+                    // single-block CTA has per-slot barriers instead.
+                    uint32_t bar, par;
+                    if (ntile == 2) {
+                        const int pt = l & 1, pi = (l - 2) >> 1;
+                        bar = is_v ? bars.pv_done(pt) : bars.s_full(pt);
+                        par = static_cast<uint32_t>(pi & 1);
+                    } else {
+                        bar = empty(st);
+                        par = static_cast<uint32_t>(((l / nst) - 1) & 1);
+                    }
+                    if (!mbar_wait(bar, par, abort_flag, WAIT_LIMIT_NS)) break;
+                }
                 mbar_arrive_expect_tx(full(st), L::TILE);
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
@@ -228,7 +249,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                     const uint64_t bd = smem_desc_sw128(sbase + L::OFF_K + st * L::TILE + off, 16);
                     mma_bf16_ss(d, ad, bd, ID_S, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bars.k_empty(st));
+                if (!has_b) mma_commit(bars.k_empty(st));
                 mma_commit(bars.s_full(t));
                 ++kl;
                 return true;
@@ -247,7 +268,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                     mma_bf16_ts(tmem + L::TMEM_O + t * 128, at, bd, ID_PV,
                                 (i > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(bars.v_empty(st));
+                if (!has_b) mma_commit(bars.v_empty(st));
                 mma_commit(bars.pv_done(t));
                 ++vl;
                 return true;

@@ -16,7 +16,7 @@
 //               s' = s + alpha * count / T on covered query blocks, then
 //               selects exactly the (topk - m) largest s' over the past blocks (equal s': smaller index
 //               first) by bitwise bisection on order-preserving keys held in
-//               registers (radix select beyond 4096 blocks), then the m
+//               registers across a CTA (radix select beyond 4096 blocks), then the m
 //               current-chunk blocks; ascending indices.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -143,10 +143,7 @@ __device__ __forceinline__ void warp_pool(const TIn* __restrict__ blk, int lane,
 // (kb = blockIdx.x * WARPS + warp, strided by the grid), pools one block at a
 // time and scores it against every query block of its head straight from
 // shared memory. Warps never wait for one another after the q-bar load.
-// CACHED: the pooled key blocks come from a k-bar cache filled by
-// kbar_append_kernel (same pooling code, so the values are bit-identical)
-// instead of being pooled from K here.
-template <typename TIn, int D, int T, bool CACHED>
+template <typename TIn, int D, int T>
 __global__ void __launch_bounds__(POOL_THREADS)
     pool_score_kernel(const TIn* __restrict__ k, const float* __restrict__ qbar, RouteArgs r) {
     using V = VecTraits<TIn>;
@@ -167,20 +164,7 @@ __global__ void __launch_bounds__(POOL_THREADS)
     float* srow = r.scores + static_cast<size_t>(bh) * r.m * r.n_past;
     for (int kb = blockIdx.x * WARPS + warp; kb < r.n_past; kb += gridDim.x * WARPS) {
         float kv[V::VEC];
-        if constexpr (CACHED) {
-            const float4* src = reinterpret_cast<const float4*>(
-                r.kbar + (static_cast<size_t>(bh) * r.kbar_cap + kb) * D + cg * V::VEC);
-#pragma unroll
-            for (int i = 0; i < V::VEC / 4; ++i) {
-                const float4 x = __ldg(src + i);
-                kv[4 * i + 0] = x.x;
-                kv[4 * i + 1] = x.y;
-                kv[4 * i + 2] = x.z;
-                kv[4 * i + 3] = x.w;
-            }
-        } else {
-            warp_pool<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, kv);
-        }
+        warp_pool<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, kv);
         // every lane runs the same number of iterations (full-warp shuffles)
         for (int q0 = 0; q0 < r.m; q0 += RPW) {
             const int qb = q0 + r0;
@@ -222,6 +206,63 @@ __global__ void __launch_bounds__(POOL_THREADS)
 #pragma unroll
         for (int j = 0; j < V::VEC / 4; ++j)
             dst[j] = make_float4(kv[4 * j], kv[4 * j + 1], kv[4 * j + 2], kv[4 * j + 3]);
+    }
+}
+
+// Scores of the past key blocks from the k-bar cache: one thread per (qb, kb)
+// output, its dot product summed in exactly the order pool_score_kernel uses
+// (per column group of VEC an FMA chain, then the pairwise tree its shuffles
+// form), so cached and streaming routing give bit-identical scores.
+constexpr int SC_KT = 64;  // key blocks per CTA
+
+template <typename TIn, int D>
+__global__ void __launch_bounds__(256) score_cached_kernel(const float* __restrict__ qbar, RouteArgs r) {
+    using V = VecTraits<TIn>;
+    constexpr int TPR = D / V::VEC;
+    extern __shared__ float sm[];
+    constexpr int KP = D + 4;          // padded row: 16-byte aligned, 128-bit reads conflict-free
+    float* q_s = sm;                   // [m][D]
+    float* k_s = q_s + r.m * D;        // [SC_KT][KP]
+    const int bh = blockIdx.y;
+    const int kb0 = blockIdx.x * SC_KT;
+    const int nk = min(SC_KT, r.n_past - kb0);
+    const int t = threadIdx.x;
+    // 16-byte loads, all of a thread's in flight together (D is a multiple of 4)
+    const float4* qsrc = reinterpret_cast<const float4*>(qbar + static_cast<size_t>(bh) * r.m * D);
+    const float4* ksrc = reinterpret_cast<const float4*>(r.kbar + (static_cast<size_t>(bh) * r.kbar_cap + kb0) * D);
+    constexpr int D4 = D / 4;
+#pragma unroll 4
+    for (int i = t; i < r.m * D4; i += 256) reinterpret_cast<float4*>(q_s)[i] = __ldg(qsrc + i);
+#pragma unroll 8
+    for (int i = t; i < nk * D4; i += 256)
+        *reinterpret_cast<float4*>(k_s + (i / D4) * KP + (i % D4) * 4) = __ldg(ksrc + i);
+    __syncthreads();
+    float* srow = r.scores + static_cast<size_t>(bh) * r.m * r.n_past + kb0;
+    for (int o = t; o < r.m * SC_KT; o += 256) {
+        const int qb = o / SC_KT, j = o % SC_KT;
+        if (j >= nk) continue;
+        const float4* qr = reinterpret_cast<const float4*>(q_s + qb * D);
+        const float4* kr = reinterpret_cast<const float4*>(k_s + j * KP);
+        float part[TPR];
+#pragma unroll
+        for (int g = 0; g < TPR; ++g) {
+            float p = 0.f;
+#pragma unroll
+            for (int v4 = 0; v4 < V::VEC / 4; ++v4) {
+                const float4 a = qr[g * (V::VEC / 4) + v4], b = kr[g * (V::VEC / 4) + v4];
+                p = fmaf(a.x, b.x, p);
+                p = fmaf(a.y, b.y, p);
+                p = fmaf(a.z, b.z, p);
+                p = fmaf(a.w, b.w, p);
+            }
+            part[g] = p;
+        }
+#pragma unroll
+        for (int w = 1; w < TPR; w <<= 1) {
+#pragma unroll
+            for (int g = 0; g < TPR; g += 2 * w) part[g] = part[g] + part[g + w];
+        }
+        srow[static_cast<size_t>(qb) * r.n_past + j] = part[0] * r.inv_sqrt_d;
     }
 }
 
@@ -270,7 +311,6 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 constexpr int SEL_WARPS = 8;
-constexpr int SEL_REG_WARPS = 4;
 
 __global__ void __launch_bounds__(SEL_WARPS * 32) select_kernel(const SelArgs a) {
     __shared__ uint32_t hist_all[SEL_WARPS][256];
@@ -354,61 +394,80 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_kernel(const SelArgs a)
     }
 }
 
-// Register-resident selection for rows of at most 32 * CH past blocks: lane l
-// keeps the keys of blocks l, l + 32, ... ; the (k_past)-th largest key is found
-// bit by bit from the top (largest u with count(key >= u) >= k_past: 32
-// rounds of compares and a warp popcount), then a ballot pass emits every
-// larger key and the first equal ones in index order. Padding keys are 0,
-// below every real key.
+// One CTA (SEL_CTA_THREADS threads) per (b, h, qb) row of at most
+// SEL_CTA_THREADS * CH past blocks: thread t keeps the keys of blocks
+// t, t + SEL_CTA_THREADS, ... in registers. The (k_past)-th largest key is found
+// bit by bit from the top (largest u with count(key >= u) >= k_past: 32 rounds
+// of compares, a warp reduction and a CTA reduction through shared memory);
+// then warp 0 emits every larger key and the first equal ones in index order
+// from a shared-memory copy of the row. Padding keys are 0, below every real key.
+constexpr int SEL_CTA_THREADS = 256;
+
 template <int CH>
-__global__ void __launch_bounds__(SEL_REG_WARPS * 32)
-    select_reg_kernel(const SelArgs a) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row = blockIdx.x * SEL_REG_WARPS + warp;
-    if (row >= a.rows) return;
+__global__ void __launch_bounds__(SEL_CTA_THREADS) select_cta_kernel(const SelArgs a) {
+    extern __shared__ uint32_t keys_s[];  // [n_past]
+    __shared__ int part[2][SEL_CTA_THREADS / 32];
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int row = blockIdx.x;
     const int n_past = a.n_past, m = a.m, k_past = a.k_past;
     const float* sc = a.scores + static_cast<size_t>(row) * n_past;
     int32_t* out = a.idx + static_cast<size_t>(row) * a.topk;
-    const RowMod mod = row_mod(a, row, lane);
-    for (int i = lane; i < m; i += 32) out[k_past + i] = n_past + i;
-    if (k_past <= 0) return;
+    for (int i = t; i < m; i += SEL_CTA_THREADS) out[k_past + i] = n_past + i;
+    if (k_past <= 0) return;  // uniform across the CTA
     if (k_past >= n_past) {
-        for (int i = lane; i < n_past; i += 32) out[i] = i;
+        for (int i = t; i < n_past; i += SEL_CTA_THREADS) out[i] = i;
         return;
     }
-    const unsigned FULL = 0xffffffffu;
+    RowMod mod{nullptr, a.alpha, a.invT, 1.0f / static_cast<float>(a.m)};
+    if (warp == 0) {
+        const RowMod w = row_mod(a, row, lane);
+        if (lane == 0) part[0][0] = w.cnt ? 1 : 0;
+    }
+    __syncthreads();
+    if (part[0][0] && a.counts) {
+        const int qb = row % a.m;
+        const int b = (row / a.m) / a.H;
+        mod.cnt = a.counts + (static_cast<size_t>(b) * a.m + qb) * a.P;
+    }
     uint32_t key[CH];
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-        const int i = c * 32 + lane;
+        const int i = c * SEL_CTA_THREADS + t;
         key[c] = i < n_past ? order_key(mod(__ldg(sc + i), i)) : 0u;
+        if (i < n_past) keys_s[i] = key[c];
     }
     uint32_t u = 0;
 #pragma unroll 1
     for (int bit = 31; bit >= 0; --bit) {
         const uint32_t cand = u | (1u << bit);
-        int c4[4] = {0, 0, 0, 0};  // independent partial counts
+        int cnt = 0;
 #pragma unroll
-        for (int c = 0; c < CH; ++c) c4[c & 3] += key[c] >= cand ? 1 : 0;
-        int cnt = (c4[0] + c4[1]) + (c4[2] + c4[3]);
+        for (int c = 0; c < CH; ++c) cnt += key[c] >= cand ? 1 : 0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o);
-        if (cnt >= k_past) u = cand;
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        const int buf = bit & 1;  // double-buffered partials: one barrier per round
+        if (lane == 0) part[buf][warp] = cnt;
+        __syncthreads();
+        int tot = 0;
+#pragma unroll
+        for (int w = 0; w < SEL_CTA_THREADS / 32; ++w) tot += part[buf][w];
+        if (tot >= k_past) u = cand;
     }
+    if (warp != 0) return;
+    const unsigned FULL = 0xffffffffu;
+    const unsigned lt = (1u << lane) - 1u;
     int gt = 0;
-#pragma unroll
-    for (int c = 0; c < CH; ++c) gt += key[c] > u ? 1 : 0;
+    for (int i = lane; i < n_past; i += 32) gt += keys_s[i] > u ? 1 : 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(FULL, gt, o);
     const int remaining = k_past - gt;
-    const unsigned lt = (1u << lane) - 1u;
     int written = 0, eq_seen = 0;
-#pragma unroll
-    for (int c = 0; c < CH; ++c) {
-        const int i = c * 32 + lane;
-        const bool eq = i < n_past && key[c] == u;
+    for (int base = 0; base < n_past; base += 32) {
+        const int i = base + lane;
+        const uint32_t k = i < n_past ? keys_s[i] : 0u;
+        const bool eq = i < n_past && k == u;
         const unsigned eqb = __ballot_sync(FULL, eq);
-        const bool take = (key[c] > u) || (eq && (eq_seen + __popc(eqb & lt)) < remaining);
+        const bool take = (k > u) || (eq && (eq_seen + __popc(eqb & lt)) < remaining);
         const unsigned tb = __ballot_sync(FULL, take);
         if (take) out[written + __popc(tb & lt)] = i;
         written += __popc(tb);
@@ -417,17 +476,18 @@ __global__ void __launch_bounds__(SEL_REG_WARPS * 32)
 }
 
 int select_launch(const SelArgs& a, cudaStream_t st) {
-    const dim3 grid((a.rows + SEL_REG_WARPS - 1) / SEL_REG_WARPS), block(SEL_REG_WARPS * 32);
-    if (a.n_past <= 32 * 2)
-        select_reg_kernel<2><<<grid, block, 0, st>>>(a);
-    else if (a.n_past <= 32 * 8)
-        select_reg_kernel<8><<<grid, block, 0, st>>>(a);
-    else if (a.n_past <= 32 * 32)
-        select_reg_kernel<32><<<grid, block, 0, st>>>(a);
-    else if (a.n_past <= 32 * 64)
-        select_reg_kernel<64><<<grid, block, 0, st>>>(a);
-    else if (a.n_past <= 32 * 128)
-        select_reg_kernel<128><<<grid, block, 0, st>>>(a);
+    const size_t smem = static_cast<size_t>(a.n_past) * sizeof(uint32_t);
+    const dim3 grid(a.rows), block(SEL_CTA_THREADS);
+    if (a.n_past <= SEL_CTA_THREADS * 1)
+        select_cta_kernel<1><<<grid, block, smem, st>>>(a);
+    else if (a.n_past <= SEL_CTA_THREADS * 2)
+        select_cta_kernel<2><<<grid, block, smem, st>>>(a);
+    else if (a.n_past <= SEL_CTA_THREADS * 4)
+        select_cta_kernel<4><<<grid, block, smem, st>>>(a);
+    else if (a.n_past <= SEL_CTA_THREADS * 8)
+        select_cta_kernel<8><<<grid, block, smem, st>>>(a);
+    else if (a.n_past <= SEL_CTA_THREADS * 16)
+        select_cta_kernel<16><<<grid, block, smem, st>>>(a);
     else
         select_kernel<<<(a.rows + SEL_WARPS - 1) / SEL_WARPS, SEL_WARPS * 32, 0, st>>>(a);
     return VELOX_OK;
@@ -439,8 +499,19 @@ int route_typed(const TIn* q, const TIn* k, const RouteArgs& r, cudaStream_t st)
     const int BH = r.B * r.H;
     pool_q_kernel<TIn, D, T><<<BH * r.m, POOL_THREADS, 0, st>>>(q, r.qbar);
     if (r.n_past > 0) {
+        if (r.kbar) {
+            const size_t smem =
+                (static_cast<size_t>(r.m) * D + static_cast<size_t>(SC_KT) * (D + 4)) * sizeof(float);
+            auto sk = score_cached_kernel<TIn, D>;
+            if (smem > 227 * 1024) return VELOX_EUNSUPPORTED;
+            if (smem > 48 * 1024 &&
+                cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)) != cudaSuccess)
+                return VELOX_ECUDA;
+            sk<<<dim3((r.n_past + SC_KT - 1) / SC_KT, BH), 256, smem, st>>>(r.qbar, r);
+        } else {
         const size_t smem = static_cast<size_t>(r.m) * D * sizeof(float);
-        auto kern = r.kbar ? pool_score_kernel<TIn, D, T, true> : pool_score_kernel<TIn, D, T, false>;
+        auto kern = pool_score_kernel<TIn, D, T>;
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
@@ -453,6 +524,7 @@ int route_typed(const TIn* q, const TIn* k, const RouteArgs& r, cudaStream_t st)
         int gx = (4 * sms + BH - 1) / BH;
         gx = max(1, min(gx, (r.n_past + warps - 1) / warps));
         kern<<<dim3(gx, BH), POOL_THREADS, smem, st>>>(k, r.qbar, r);
+        }
     }
     // the counts are read by the selection only: it may wait for them alone
     if (r.counts_ready && cudaStreamWaitEvent(st, r.counts_ready, 0) != cudaSuccess)
