@@ -1,7 +1,7 @@
 """Benchmark of the Velox geometry-routed attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload headline|sweep] [--P 48]
+                    [--workload headline|sweep|pipeline|robustness] [--P 48]
 
 One step = one pass of the whole hot path over one chunk's synthetic inputs,
 with the KV cache resident in HBM: frustum slices of every past chunk, slice
@@ -19,6 +19,13 @@ collective -- and the time is the max over ranks ("scaling": "weak").
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload (the oracle stands in for a reference
 implementation: the method's pages publish no code).
+
+--workload robustness (one GPU) measures how depth-estimation error moves
+the selection: at P = 48, 96, 192 and 224 past chunks (or --P) the routing
+from ground-truth depth is compared, row by row, with the routing of the
+full geometry pipeline (multiwarp -> slices -> overlap) fed with perturbed
+past depth (scale bias, multiplicative noise, holes); it also times routing,
+sparse and dense attention at each P.
 """
 from __future__ import annotations
 
@@ -629,6 +636,138 @@ def run_pipeline(args):
         print(json.dumps(out), flush=True)
 
 
+ROBUST_P = (48, 96, 192, 224)
+DEPTH_ERRORS = (
+    ("none", {}),
+    ("scale x0.8", {"scale": 0.8}), ("scale x0.9", {"scale": 0.9}),
+    ("scale x1.1", {"scale": 1.1}), ("scale x1.25", {"scale": 1.25}),
+    ("noise 2%", {"noise_sd": 0.02}), ("noise 5%", {"noise_sd": 0.05}),
+    ("noise 10%", {"noise_sd": 0.10}), ("noise 20%", {"noise_sd": 0.20}),
+    ("holes 10%", {"hole_frac": 0.10}), ("holes 30%", {"hole_frac": 0.30}),
+    ("holes 50%", {"hole_frac": 0.50}),
+)
+
+
+def selection_change(ref: np.ndarray, got: np.ndarray, n_past: int) -> dict:
+    """Rows of ascending key-block lists [..., k]: how the past blocks `got`
+    keeps differ from those `ref` keeps (current-chunk blocks, always kept,
+    are left out). Mean Jaccard index and recall of `ref`'s blocks, and the
+    fraction of rows whose past sets are identical."""
+    ref = ref.reshape(-1, ref.shape[-1])
+    got = got.reshape(-1, got.shape[-1])
+    R = ref.shape[0]
+    a = np.zeros((R, n_past), dtype=bool)
+    b = np.zeros((R, n_past), dtype=bool)
+    for mask, lst in ((a, ref), (b, got)):
+        rows = np.broadcast_to(np.arange(R)[:, None], lst.shape)
+        keep = lst < n_past
+        mask[rows[keep], lst[keep]] = True
+    inter = (a & b).sum(1)
+    union = (a | b).sum(1)
+    na = a.sum(1)
+    jac = np.where(union > 0, inter / np.maximum(union, 1), 1.0)
+    rec = np.where(na > 0, inter / np.maximum(na, 1), 1.0)
+    return {"jaccard": round(float(jac.mean()), 4), "recall": round(float(rec.mean()), 4),
+            "rows_identical": round(float((inter == union).mean()), 4)}
+
+
+def draw_qkv_on_device(torch, s, view_overlap, seed: int, device):
+    """Workload 3's Q/K/V structure drawn on the device, one head at a time
+    (bounded temporaries at any P): Q = N(0,1) + mu_h, past chunk c's K =
+    N(0,1) + view_overlap[c] * mu_h, current K and V = N(0,1)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    mu = 0.5 * torch.randn((s.H, s.d), generator=g, device=device)
+    ov = torch.tensor(np.asarray(view_overlap), dtype=torch.float32, device=device)
+    q = torch.empty((s.B, s.H, s.Nq, s.d), dtype=torch.bfloat16, device=device)
+    k = torch.empty((s.B, s.H, s.Nk, s.d), dtype=torch.bfloat16, device=device)
+    v = torch.empty((s.B, s.H, s.Nk, s.d), dtype=torch.bfloat16, device=device)
+    for b in range(s.B):
+        for h in range(s.H):
+            q[b, h] = torch.randn((s.Nq, s.d), generator=g, device=device) + mu[h]
+            kh = torch.randn((s.P + 1, s.Nq, s.d), generator=g, device=device)
+            kh[: s.P] += ov.view(s.P, 1, 1) * mu[h].view(1, 1, s.d)
+            k[b, h] = kh.view(s.Nk, s.d)
+            del kh
+            v[b, h] = torch.randn((s.Nk, s.d), generator=g, device=device)
+    return q, k, v
+
+
+def run_robustness(args):
+    import torch
+    from geometry_routed_block_b200 import velox as vx
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    reps = max(3, min(args.steps, 10))
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    per_p = []
+    for P in ([args.P] if args.P else ROBUST_P):
+        geo = synth.geometry_only(4, P=P)
+        s = synth.shape_for(4, P=P)
+        q, k, v = draw_qkv_on_device(torch, s, geo.meta["view_overlap"], 1004 + P, device)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        past_poses, past_intr = dev(geo.past_poses[0]), dev(geo.past_intr[0])
+        past_cams, cur_cam = dev(geo.past_cams[0]), dev(geo.cur_cam)
+        mw_ws = vx.depth_multiwarp_workspace(s.Hp, s.Wp, device)
+        ws = vx.route_workspace(s.B, s.H, s.Nq, s.Nk, s.d, s.T, device)
+        n_past = s.P * s.m
+
+        def counts_for(past_depth, cur_depth):
+            sl = vx.slices_build(past_depth, past_poses, past_intr)
+            return vx.block_overlap(cur_depth, cur_cam, sl[None], s.F, s.T)
+
+        def route(counts):
+            return vx.route_topk(q, k, counts, s.alpha, s.topk, s.T, ws=ws).cpu().numpy()
+
+        gt_counts = counts_for(dev(geo.past_depth[0]), dev(geo.cur_depth))
+        gtc = gt_counts.cpu().numpy()
+        idx_gt = route(gt_counts)
+        rows = [{"depth_error": "no geometry (alpha = 0)",
+                 **selection_change(idx_gt, route(None), n_past)}]
+        for e, (name, kw) in enumerate(DEPTH_ERRORS):
+            rng = np.random.default_rng([1004, P, e])
+            past = synth.perturb_depth(geo.past_depth[0], rng, **kw) if kw else geo.past_depth[0]
+            past_t = dev(past)
+            cur = vx.depth_multiwarp(past_t, past_cams, cur_cam[0], 0.01, ws=mw_ws)
+            counts = counts_for(past_t, cur[None])
+            c = counts.cpu().numpy()
+            rows.append({"depth_error": name + " (multiwarp current depth)",
+                         **selection_change(idx_gt, route(counts), n_past),
+                         "count_mae_over_T": round(float(np.abs(c - gtc).mean()) / s.T, 4),
+                         "covered_query_blocks": int((c.sum(-1) > 0).sum())})
+        # timing at this P on the ground-truth route
+        idx = torch.from_numpy(idx_gt).to(device)
+        o, o2 = torch.empty_like(q), torch.empty_like(q)
+        route_dev = lambda: vx.route_topk(q, k, gt_counts, s.alpha, s.topk, s.T, ws=ws, out=idx)
+        attend = lambda: vx.sparse_attn_fwd(q, k, v, idx, s.T, out=o, want_lse=False, status=status)
+        dense = lambda: vx.sparse_attn_fwd(q, k, v, None, s.T, out=o2, want_lse=False, status=status)
+        for _ in range(3):
+            route_dev()
+            attend()
+        dense()
+        t_route = time_loop(torch, route_dev, reps)
+        t_attn = time_loop(torch, attend, reps)
+        t_dense = time_loop(torch, dense, 2)
+        per_p.append({
+            "P": P, "key_blocks": s.nKB, "topk": s.topk, "covered_query_blocks_gt":
+            int((gtc.sum(-1) > 0).sum()), "selection_vs_ground_truth_depth": rows,
+            "routing_ms": round(t_route, 4), "routing_gbs": round(routing_bytes(s) / t_route / 1e6, 1),
+            "sparse_attn_ms": round(t_attn, 4),
+            "sparse_attn_tflops": round(kept_flops(s) / t_attn / 1e9, 1),
+            "dense_attn_ms": round(t_dense, 4),
+            "speedup_vs_dense": round(t_dense / (t_route + t_attn), 3),
+        })
+        del q, k, v, o, o2, ws
+        torch.cuda.empty_cache()
+    out = {"workload": "robustness: depth error vs selection, rollouts P = "
+           + "/".join(str(r["P"]) for r in per_p) + " (B1 H24 d128 T128, 3x32x48 chunks, k = 20%)",
+           "data": "synthetic", "n_gpus": 1, "device_status": int(status.item()), "per_P": per_p}
+    print(json.dumps(out), flush=True)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -671,7 +810,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
-    ap.add_argument("--workload", default="headline", choices=["headline", "sweep", "pipeline"])
+    ap.add_argument("--workload", default="headline",
+                    choices=["headline", "sweep", "pipeline", "robustness"])
     ap.add_argument("--layers", type=int, default=30, help="layers (pipeline workload)")
     ap.add_argument("--P", type=int, default=None, help="past chunks (sweep workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -680,6 +820,8 @@ def main():
         run_reference(args)
     elif args.workload == "pipeline":
         run_pipeline(args)
+    elif args.workload == "robustness":
+        run_robustness(args)
     else:
         run_gpu(args)
 

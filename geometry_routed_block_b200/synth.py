@@ -394,6 +394,21 @@ def _loop(cfg: int, seed: int, s: Shape, heads: tuple | None = None) -> Case:
                 meta={"view_overlap": ov, "heads": hsel})
 
 
+def perturb_depth(depth: np.ndarray, rng: np.random.Generator, noise_sd: float = 0.0,
+                  hole_frac: float = 0.0, scale: float = 1.0) -> np.ndarray:
+    """Depth-estimation error model for robustness studies (input generation,
+    not a step of the method): a global scale bias, then per-pixel
+    multiplicative Gaussian noise z * (1 + noise_sd * N(0,1)), then holes (NaN)
+    at a random `hole_frac` of the pixels. Pixels that were invalid stay
+    invalid; noise that drives a depth to <= 0 leaves it invalid as well."""
+    d = np.asarray(depth, dtype=np.float64) * scale
+    if noise_sd > 0:
+        d = d * (1.0 + noise_sd * rng.standard_normal(d.shape))
+    if hole_frac > 0:
+        d[rng.random(d.shape) < hole_frac] = np.nan
+    return d.astype(np.float32)
+
+
 def make_case(cfg: int, seed: int | None = None, P: int | None = None, H: int | None = None,
               layers: int | None = None, heads: tuple | None = None) -> Case:
     """Build workload `cfg` (1..5). Default seed is 1000 + cfg."""

@@ -288,6 +288,30 @@ def test_rollout_p96_routing_sampled_heads(vx):
     assert compare_selection(idx.cpu().numpy(), want, s_mod, s.m) <= 3
 
 
+def test_rollout_p224_largest_size_geometry_routing_attention(vx):
+    """224 past chunks: 8,100 key blocks (the router's limit is 8,192), 8,064
+    past candidates per row (the radix selection path), 1,620 kept blocks."""
+    c = synth.make_case(4, P=224, heads=(5,))
+    s = c.shape
+    assert s.nKB == 8100 and s.topk == 1620
+    sl = vx.slices_build(dev(c.past_depth[0]), dev(c.past_poses[0]), dev(c.past_intr[0]))
+    want_sl = vo.slices_build(c.past_depth[0], c.past_poses[0], c.past_intr[0])
+    assert np.array_equal(sl.cpu().numpy(), want_sl)
+    counts = vo.block_overlap(c.cur_depth, c.cur_cam, want_sl[None], s.F, s.T)
+    got_counts = vx.block_overlap(dev(c.cur_depth), dev(c.cur_cam), sl[None], s.F, s.T)
+    assert np.array_equal(got_counts.cpu().numpy(), counts)
+    q, k, v = dev(c.q[0]), dev(c.k[0]), dev(c.v[0])
+    idx = vx.route_topk(q, k, got_counts, s.alpha, s.topk, s.T)
+    want, s_mod = vo.route_topk(c.q[0], c.k[0], counts, s.alpha, s.topk, s.T)
+    assert compare_selection(idx.cpu().numpy(), want, s_mod, s.m) <= 3
+    o, lse = vx.sparse_attn_fwd(q, k, v, dev(want), s.T)
+    ref = vo.sparse_attention(c.q[0], c.k[0], c.v[0], want, s.T, rows=[(0, 0, 0), (0, 0, 35)])
+    for (b, h, qb), (o_ref, lse_ref) in ref.items():
+        sl_ = slice(qb * s.T, (qb + 1) * s.T)
+        compare_attention(o[b, h, sl_], o_ref, f"P=224 row {(b, h, qb)}")
+        assert np.abs(lse[b, h, sl_].cpu().numpy() - lse_ref).max() < 1e-3
+
+
 def test_route_exact_ties_break_to_the_smaller_index(vx):
     # past chunks 0-2 are copies, and so are 3-5: their pooled scores tie exactly
     # (in fp32 on the device and in fp64 in the oracle), so the selection is
