@@ -1,7 +1,7 @@
 """Benchmark of the Velox geometry-routed attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload headline|sweep|pipeline|robustness] [--P 48]
+                    [--workload headline|sweep|pipeline|robustness|rollout] [--P 48]
 
 One step = one pass of the whole hot path over one chunk's synthetic inputs,
 with the KV cache resident in HBM: frustum slices of every past chunk, slice
@@ -26,6 +26,11 @@ from ground-truth depth is compared, row by row, with the routing of the
 full geometry pipeline (multiwarp -> slices -> overlap) fed with perturbed
 past depth (scale bias, multiplicative noise, holes); it also times routing,
 sparse and dense attention at each P.
+
+--workload rollout runs --chunks consecutive chunks from --P, each denoised
+in --denoise-steps steps of --layers layers (pooled-key-cache routing and
+sparse attention over a KV cache sized for all of them), with the geometry
+built at each chunk boundary or pipelined one chunk ahead.
 """
 from __future__ import annotations
 
@@ -768,6 +773,114 @@ def run_robustness(args):
     print(json.dumps(out), flush=True)
 
 
+def run_rollout(args):
+    """Several consecutive chunks of a rollout, each denoised in S steps of L
+    layers: pooled-key-cache routing + sparse attention per layer, the pooled
+    keys of a chunk appended when it is done, and the geometry either built
+    at each chunk boundary or pipelined one chunk ahead. Reports both
+    schedules' time per chunk and how much the look-ahead geometry (built from
+    the previous chunk's warped depth, its final depth not yet known) changes
+    the selection."""
+    import torch
+    from geometry_routed_block_b200 import velox as vx
+    from geometry_routed_block_b200.rollout import Rollout
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    P0 = args.P or 48
+    C, S, L = args.chunks, args.denoise_steps, args.layers
+    cap = P0 + C  # chunks 0..cap-1 live in the KV cache
+    seed = 1004 + rank
+    geo = synth.geometry_only(4, seed=seed, P=cap)  # cameras and depth of chunks 0..cap
+    s = synth.shape_for(4, P=cap - 1)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    cams = dev(np.concatenate([geo.past_cams[0], geo.cur_cam], 0))
+    poses, intr = dev(geo.past_poses[0]), dev(geo.past_intr[0])
+    final_depth = dev(np.concatenate([geo.past_depth[0], geo.cur_depth], 0))
+    ov = np.asarray(geo.meta["view_overlap"])[: cap - 1]
+    qs, ks, vs = [], [], []
+    for layer in range(L):
+        q, k, v = draw_qkv_on_device(torch, s, ov, seed * 1000 + layer, device)
+        qs.append(q), ks.append(k), vs.append(v)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    o = torch.empty_like(qs[0])
+    topk_of = lambda n: synth.topk_for(n, s.m)
+    idx_buf = {n: torch.empty((s.B, s.H, s.m, topk_of(n)), dtype=torch.int32, device=device)
+               for n in range(P0, cap)}
+    states = {}
+    for sched in ("boundary", "pipelined"):
+        R = Rollout(ks, B=s.B, H=s.H, d=s.d, T=s.T, F=s.F, Hp=s.Hp, Wp=s.Wp, capacity=cap,
+                    cams=cams, poses=poses, intr=intr, alpha=s.alpha, topk_of=topk_of,
+                    schedule=sched)
+        R.prefill(P0, final_depth[:P0])
+        states[sched] = R
+
+    def rollout(R, marks=None):
+        for n in range(P0, cap):
+            if marks is not None:
+                marks[n][0].record()
+            R.begin_chunk(n)
+            for step in range(S):
+                for layer in range(L):
+                    idx = R.route(layer, qs[layer], out=idx_buf[n])
+                    if marks is not None and step == 0 and layer == 0:
+                        marks[n][1].record()
+                    R.attend(layer, qs[layer], vs[layer], idx, out=o, status=status)
+            R.end_chunk(n, final_depth[n])
+
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    times = {k: [] for k in states}
+    first_route = {k: [] for k in states}
+    reps = max(1, min(args.steps, 3))
+    for it in range(1 + reps):  # one untimed rollout per schedule, then interleaved reps
+        for sched, R in states.items():
+            R.start(P0)
+            torch.cuda.synchronize()
+            marks = {n: (mk(), mk()) for n in range(P0, cap)}
+            a, b = mk(), mk()
+            a.record()
+            rollout(R, marks)
+            b.record()
+            torch.cuda.synchronize()
+            if it > 0:
+                times[sched].append(a.elapsed_time(b) / C)
+                first_route[sched] += [marks[n][0].elapsed_time(marks[n][1])
+                                       for n in range(P0, cap)]
+    med = statistics.median
+    t = reduce_max([med(times["boundary"]), med(times["pipelined"])], device)
+    # selection change of the look-ahead geometry: layer 0 of every chunk
+    rows = []
+    Rb, Rp = states["boundary"], states["pipelined"]
+    for n in range(P0, cap):
+        ib = vx.route_topk_cached(qs[0], Rb.kbar[0], n, Rb.counts[n], s.alpha, topk_of(n), s.T)
+        ip = vx.route_topk_cached(qs[0], Rp.kbar[0], n, Rp.counts[n], s.alpha, topk_of(n), s.T)
+        cb, cp = Rb.counts[n].cpu().numpy(), Rp.counts[n].cpu().numpy()
+        rows.append({"chunk": n, **selection_change(ib.cpu().numpy(), ip.cpu().numpy(), n * s.m),
+                     "count_mae_over_T": round(float(np.abs(cb - cp).mean()) / s.T, 4)})
+    kf = sum(S * L * 4.0 * s.B * s.H * s.m * topk_of(n) * s.T * s.T * s.d for n in range(P0, cap))
+    value = world * kf / (t[1] * C * 1e-3) / 1e12
+    launches_chunk = S * L * 4 + L + 8  # route (3) + attention per layer; appends; geometry
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": reps, "warmup": 1, "ms_per_step": round(t[1] * C, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"rollout of chunks {P0}..{cap - 1}, {S} denoising steps x {L} "
+                   f"layers per chunk, pooled-key-cache routing, KV cache of {cap} chunks; "
+                   + workload_desc(s), "l2": "inputs larger than L2; no flush"},
+        "chunk_ms": {"boundary": round(t[0], 3), "pipelined": round(t[1], 3)},
+        "geometry_exposed_ms_per_chunk": round(t[0] - t[1], 4),
+        "first_route_done_ms": {k: round(med(v), 4) for k, v in first_route.items()},
+        "lookahead_selection_vs_boundary": rows,
+        "gpu_launches": launches_chunk * C * reps,
+        "device_status": int(status.item()),
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -811,7 +924,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
     ap.add_argument("--workload", default="headline",
-                    choices=["headline", "sweep", "pipeline", "robustness"])
+                    choices=["headline", "sweep", "pipeline", "robustness", "rollout"])
+    ap.add_argument("--chunks", type=int, default=4, help="chunks (rollout workload)")
+    ap.add_argument("--denoise-steps", type=int, default=4, help="steps per chunk (rollout)")
     ap.add_argument("--layers", type=int, default=30, help="layers (pipeline workload)")
     ap.add_argument("--P", type=int, default=None, help="past chunks (sweep workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -822,6 +937,8 @@ def main():
         run_pipeline(args)
     elif args.workload == "robustness":
         run_robustness(args)
+    elif args.workload == "rollout":
+        run_rollout(args)
     else:
         run_gpu(args)
 
