@@ -394,28 +394,34 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_kernel(const SelArgs a)
     }
 }
 
-// One CTA (SEL_CTA_THREADS threads) per (b, h, qb) row of at most
-// SEL_CTA_THREADS * CH past blocks: thread t keeps the keys of blocks
-// t, t + SEL_CTA_THREADS, ... in registers. The (k_past)-th largest key is found
-// bit by bit from the top (largest u with count(key >= u) >= k_past: 32 rounds
-// of compares, a warp reduction and a CTA reduction through shared memory);
-// then warp 0 emits every larger key and the first equal ones in index order
-// from a shared-memory copy of the row. Padding keys are 0, below every real key.
-constexpr int SEL_CTA_THREADS = 256;
+// One CTA (THREADS threads) per (b, h, qb) row of at most THREADS * CH past
+// blocks: thread t keeps the keys of blocks t, t + THREADS, ... in registers.
+// The (k_past)-th largest key u is found bit by bit from the top (largest u
+// with count(key >= u) >= k_past), starting below the common prefix of the
+// row's smallest and largest keys (u lies between them); each round is a warp
+// reduction and one CTA barrier.
+// Then every warp emits, from a shared-memory copy of its segment of the row,
+// the keys above u and the first equal ones in index order, at offsets from a
+// prefix over the warps' counts. Padding keys are 0, below every real key.
+constexpr int SEL_CTA_THREADS = 256;  // measured against 64 and 128
 
-template <int CH>
-__global__ void __launch_bounds__(SEL_CTA_THREADS) select_cta_kernel(const SelArgs a) {
+template <int THREADS, int CH>
+__global__ void __launch_bounds__(THREADS) select_cta_kernel(const SelArgs a) {
+    constexpr int SEL_CTA_WARPS = THREADS / 32;
     extern __shared__ uint32_t keys_s[];  // [n_past]
-    __shared__ int part[2][SEL_CTA_THREADS / 32];
+    __shared__ __align__(16) int part[2][SEL_CTA_WARPS];
+    __shared__ uint32_t span[2][SEL_CTA_WARPS];
+    __shared__ int seg_cnt[2][SEL_CTA_WARPS];
+    const unsigned FULL = 0xffffffffu;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int row = blockIdx.x;
     const int n_past = a.n_past, m = a.m, k_past = a.k_past;
     const float* sc = a.scores + static_cast<size_t>(row) * n_past;
     int32_t* out = a.idx + static_cast<size_t>(row) * a.topk;
-    for (int i = t; i < m; i += SEL_CTA_THREADS) out[k_past + i] = n_past + i;
+    for (int i = t; i < m; i += THREADS) out[k_past + i] = n_past + i;
     if (k_past <= 0) return;  // uniform across the CTA
     if (k_past >= n_past) {
-        for (int i = t; i < n_past; i += SEL_CTA_THREADS) out[i] = i;
+        for (int i = t; i < n_past; i += THREADS) out[i] = i;
         return;
     }
     RowMod mod{nullptr, a.alpha, a.invT, 1.0f / static_cast<float>(a.m)};
@@ -430,44 +436,83 @@ __global__ void __launch_bounds__(SEL_CTA_THREADS) select_cta_kernel(const SelAr
         mod.cnt = a.counts + (static_cast<size_t>(b) * a.m + qb) * a.P;
     }
     uint32_t key[CH];
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-        const int i = c * SEL_CTA_THREADS + t;
+        const int i = c * THREADS + t;
         key[c] = i < n_past ? order_key(mod(__ldg(sc + i), i)) : 0u;
-        if (i < n_past) keys_s[i] = key[c];
+        if (i < n_past) {
+            keys_s[i] = key[c];
+            kmin = min(kmin, key[c]);
+            kmax = max(kmax, key[c]);
+        }
     }
-    uint32_t u = 0;
+    kmin = __reduce_min_sync(FULL, kmin);
+    kmax = __reduce_max_sync(FULL, kmax);
+    if (lane == 0) {
+        span[0][warp] = kmin;
+        span[1][warp] = kmax;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < SEL_CTA_WARPS; ++w) {
+        kmin = min(kmin, span[0][w]);
+        kmax = max(kmax, span[1][w]);
+    }
+    // bits above the highest one where min and max differ are u's already
+    const uint32_t diff = kmin ^ kmax;
+    const int top = diff ? 31 - __clz(diff) : -1;
+    uint32_t u = top < 0 ? kmax : (kmax & ~((2u << top) - 1u));
 #pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
+    for (int bit = top; bit >= 0; --bit) {
         const uint32_t cand = u | (1u << bit);
-        int cnt = 0;
+        unsigned cnt = 0;
 #pragma unroll
-        for (int c = 0; c < CH; ++c) cnt += key[c] >= cand ? 1 : 0;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        for (int c = 0; c < CH; ++c) cnt += key[c] >= cand ? 1u : 0u;
+        cnt = __reduce_add_sync(FULL, cnt);
         const int buf = bit & 1;  // double-buffered partials: one barrier per round
-        if (lane == 0) part[buf][warp] = cnt;
+        if (lane == 0) part[buf][warp] = static_cast<int>(cnt);
         __syncthreads();
         int tot = 0;
 #pragma unroll
-        for (int w = 0; w < SEL_CTA_THREADS / 32; ++w) tot += part[buf][w];
+        for (int w = 0; w < SEL_CTA_WARPS; ++w) tot += part[buf][w];
         if (tot >= k_past) u = cand;
     }
-    if (warp != 0) return;
-    const unsigned FULL = 0xffffffffu;
+    // emission: warp w owns keys [s0, s1) of the row
     const unsigned lt = (1u << lane) - 1u;
-    int gt = 0;
-    for (int i = lane; i < n_past; i += 32) gt += keys_s[i] > u ? 1 : 0;
+    const int seg = ((n_past + THREADS - 1) / THREADS) * 32;
+    const int s0 = min(n_past, warp * seg), s1 = min(n_past, s0 + seg);
+    unsigned gt = 0, eq = 0;
+    for (int i = s0 + lane; i < s1; i += 32) {
+        const uint32_t k = keys_s[i];
+        gt += k > u ? 1u : 0u;
+        eq += k == u ? 1u : 0u;
+    }
+    gt = __reduce_add_sync(FULL, gt);
+    eq = __reduce_add_sync(FULL, eq);
+    if (lane == 0) {
+        seg_cnt[0][warp] = static_cast<int>(gt);
+        seg_cnt[1][warp] = static_cast<int>(eq);
+    }
+    __syncthreads();
+    int gt_total = 0, gt_before = 0, eq_before = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(FULL, gt, o);
-    const int remaining = k_past - gt;
-    int written = 0, eq_seen = 0;
-    for (int base = 0; base < n_past; base += 32) {
+    for (int w = 0; w < SEL_CTA_WARPS; ++w) {
+        gt_total += seg_cnt[0][w];
+        if (w < warp) {
+            gt_before += seg_cnt[0][w];
+            eq_before += seg_cnt[1][w];
+        }
+    }
+    const int remaining = k_past - gt_total;  // equal keys taken, smallest indices first
+    int written = gt_before + min(eq_before, remaining);
+    int eq_seen = eq_before;
+    for (int base = s0; base < s1; base += 32) {
         const int i = base + lane;
-        const uint32_t k = i < n_past ? keys_s[i] : 0u;
-        const bool eq = i < n_past && k == u;
-        const unsigned eqb = __ballot_sync(FULL, eq);
-        const bool take = (k > u) || (eq && (eq_seen + __popc(eqb & lt)) < remaining);
+        const uint32_t k = i < s1 ? keys_s[i] : 0u;
+        const bool is_eq = i < s1 && k == u;
+        const unsigned eqb = __ballot_sync(FULL, is_eq);
+        const bool take = (i < s1 && k > u) || (is_eq && (eq_seen + __popc(eqb & lt)) < remaining);
         const unsigned tb = __ballot_sync(FULL, take);
         if (take) out[written + __popc(tb & lt)] = i;
         written += __popc(tb);
@@ -476,18 +521,19 @@ __global__ void __launch_bounds__(SEL_CTA_THREADS) select_cta_kernel(const SelAr
 }
 
 int select_launch(const SelArgs& a, cudaStream_t st) {
+    constexpr int TH = SEL_CTA_THREADS;
     const size_t smem = static_cast<size_t>(a.n_past) * sizeof(uint32_t);
-    const dim3 grid(a.rows), block(SEL_CTA_THREADS);
-    if (a.n_past <= SEL_CTA_THREADS * 1)
-        select_cta_kernel<1><<<grid, block, smem, st>>>(a);
-    else if (a.n_past <= SEL_CTA_THREADS * 2)
-        select_cta_kernel<2><<<grid, block, smem, st>>>(a);
-    else if (a.n_past <= SEL_CTA_THREADS * 4)
-        select_cta_kernel<4><<<grid, block, smem, st>>>(a);
-    else if (a.n_past <= SEL_CTA_THREADS * 8)
-        select_cta_kernel<8><<<grid, block, smem, st>>>(a);
-    else if (a.n_past <= SEL_CTA_THREADS * 16)
-        select_cta_kernel<16><<<grid, block, smem, st>>>(a);
+    const dim3 grid(a.rows), block(TH);
+    if (a.n_past <= TH * 1)
+        select_cta_kernel<TH, 1><<<grid, block, smem, st>>>(a);
+    else if (a.n_past <= TH * 2)
+        select_cta_kernel<TH, 2><<<grid, block, smem, st>>>(a);
+    else if (a.n_past <= TH * 4)
+        select_cta_kernel<TH, 4><<<grid, block, smem, st>>>(a);
+    else if (a.n_past <= TH * 8)
+        select_cta_kernel<TH, 8><<<grid, block, smem, st>>>(a);
+    else if (a.n_past <= TH * 16)
+        select_cta_kernel<TH, 16><<<grid, block, smem, st>>>(a);
     else
         select_kernel<<<(a.rows + SEL_WARPS - 1) / SEL_WARPS, SEL_WARPS * 32, 0, st>>>(a);
     return VELOX_OK;
