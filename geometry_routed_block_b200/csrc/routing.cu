@@ -209,16 +209,26 @@ __global__ void __launch_bounds__(POOL_THREADS)
     }
 }
 
-// Scores of the past key blocks from the k-bar cache: one thread per (qb, kb)
-// output, its dot product summed in exactly the order pool_score_kernel uses
-// (per column group of VEC an FMA chain, then the pairwise tree its shuffles
-// form), so cached and streaming routing give bit-identical scores.
-constexpr int SC_KT = 64;  // key blocks per CTA
+// Scores of the past key blocks from the k-bar cache, each dot product summed
+// in exactly the order pool_score_kernel uses (per column group of VEC an FMA
+// chain, then the pairwise tree its shuffles form), so cached and streaming
+// routing give bit-identical scores. A CTA takes SC_KT cached blocks of one
+// head; thread (j, g) scores block j against SC_QA query blocks at a time
+// (groups g, g + SC_QG, ...), so one shared-memory read of a key group serves
+// SC_QA outputs and the query groups are warp-wide broadcasts. The tree is
+// built as the column groups come: a node that is a right child at level L is
+// added to the left subtree kept for that level.
+constexpr int SC_KT = 32;  // key blocks per CTA
+constexpr int SC_QG = 8;   // 256 threads = SC_KT x SC_QG
+constexpr int SC_QA = 5;   // query blocks per thread and pass
 
 template <typename TIn, int D>
 __global__ void __launch_bounds__(256) score_cached_kernel(const float* __restrict__ qbar, RouteArgs r) {
     using V = VecTraits<TIn>;
-    constexpr int TPR = D / V::VEC;
+    constexpr int VEC = V::VEC;
+    constexpr int TPR = D / VEC;  // column groups = lanes of one row in the streaming scorer
+    constexpr int LOG = TPR == 8 ? 3 : (TPR == 16 ? 4 : 5);
+    static_assert((1 << LOG) == TPR, "column groups must be 8, 16 or 32");
     extern __shared__ float sm[];
     constexpr int KP = D + 4;          // padded row: 16-byte aligned, 128-bit reads conflict-free
     float* q_s = sm;                   // [m][D]
@@ -237,32 +247,66 @@ __global__ void __launch_bounds__(256) score_cached_kernel(const float* __restri
     for (int i = t; i < nk * D4; i += 256)
         *reinterpret_cast<float4*>(k_s + (i / D4) * KP + (i % D4) * 4) = __ldg(ksrc + i);
     __syncthreads();
-    float* srow = r.scores + static_cast<size_t>(bh) * r.m * r.n_past + kb0;
-    for (int o = t; o < r.m * SC_KT; o += 256) {
-        const int qb = o / SC_KT, j = o % SC_KT;
-        if (j >= nk) continue;
-        const float4* qr = reinterpret_cast<const float4*>(q_s + qb * D);
-        const float4* kr = reinterpret_cast<const float4*>(k_s + j * KP);
-        float part[TPR];
+    const int j = t % SC_KT;
+    if (j >= nk) return;  // no barrier follows
+    const float4* krow = reinterpret_cast<const float4*>(k_s + j * KP);
+    float* scol = r.scores + static_cast<size_t>(bh) * r.m * r.n_past + kb0 + j;
+    for (int q0 = (t / SC_KT) * SC_QA; q0 < r.m; q0 += SC_QG * SC_QA) {
+        float stk[SC_QA][LOG];  // [a][L]: left subtree pending at level L (L >= 1)
+        float root[SC_QA];
+#pragma unroll 1
+        for (int c = 0; c < TPR / 2; ++c) {  // column groups 2c and 2c + 1: a level-1 node
+            float node[SC_QA];
 #pragma unroll
-        for (int g = 0; g < TPR; ++g) {
-            float p = 0.f;
+            for (int h = 0; h < 2; ++h) {
+                const int g = 2 * c + h;
+                float kv[VEC];
 #pragma unroll
-            for (int v4 = 0; v4 < V::VEC / 4; ++v4) {
-                const float4 a = qr[g * (V::VEC / 4) + v4], b = kr[g * (V::VEC / 4) + v4];
-                p = fmaf(a.x, b.x, p);
-                p = fmaf(a.y, b.y, p);
-                p = fmaf(a.z, b.z, p);
-                p = fmaf(a.w, b.w, p);
+                for (int v4 = 0; v4 < VEC / 4; ++v4) {
+                    const float4 b = krow[g * (VEC / 4) + v4];
+                    kv[4 * v4] = b.x;
+                    kv[4 * v4 + 1] = b.y;
+                    kv[4 * v4 + 2] = b.z;
+                    kv[4 * v4 + 3] = b.w;
+                }
+#pragma unroll
+                for (int a = 0; a < SC_QA; ++a) {
+                    const int qb = min(q0 + a, r.m - 1);  // rows past m are computed and dropped
+                    const float4* qr = reinterpret_cast<const float4*>(q_s + qb * D + g * VEC);
+                    float p = 0.f;
+#pragma unroll
+                    for (int v4 = 0; v4 < VEC / 4; ++v4) {
+                        const float4 x = qr[v4];
+                        p = fmaf(x.x, kv[4 * v4], p);
+                        p = fmaf(x.y, kv[4 * v4 + 1], p);
+                        p = fmaf(x.z, kv[4 * v4 + 2], p);
+                        p = fmaf(x.w, kv[4 * v4 + 3], p);
+                    }
+                    node[a] = h == 0 ? p : node[a] + p;
+                }
             }
-            part[g] = p;
+            // node c at level 1 is a right child at level L when bit L-1 of c is set
+#pragma unroll
+            for (int a = 0; a < SC_QA; ++a) {
+                float v = node[a];
+                bool placed = false;
+#pragma unroll
+                for (int L = 1; L < LOG; ++L) {
+                    if (!placed) {
+                        if (((c >> (L - 1)) & 1) == 0) {
+                            stk[a][L] = v;
+                            placed = true;
+                        } else {
+                            v = stk[a][L] + v;
+                        }
+                    }
+                }
+                if (!placed) root[a] = v;
+            }
         }
 #pragma unroll
-        for (int w = 1; w < TPR; w <<= 1) {
-#pragma unroll
-            for (int g = 0; g < TPR; g += 2 * w) part[g] = part[g] + part[g + w];
-        }
-        srow[static_cast<size_t>(qb) * r.n_past + j] = part[0] * r.inv_sqrt_d;
+        for (int a = 0; a < SC_QA; ++a)
+            if (q0 + a < r.m) scol[static_cast<size_t>(q0 + a) * r.n_past] = root[a] * r.inv_sqrt_d;
     }
 }
 
