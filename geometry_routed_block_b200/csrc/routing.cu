@@ -606,13 +606,20 @@ int route_typed(const TIn* q, const TIn* k, const RouteArgs& r, cudaStream_t st)
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
             return VELOX_ECUDA;
-        int dev = 0, sms = 148;
+        int dev = 0, sms = 148, occ = 1;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        // about 4 resident CTAs per SM over all heads, never more warps than blocks
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, POOL_THREADS, smem) !=
+                cudaSuccess ||
+            occ < 1)
+            occ = 1;
+        // every CTA resident at once, and every warp with the same number of
+        // key blocks (the fewest per warp that fit, then the fewest CTAs that
+        // give it): the stream of K has no tail of half-busy SMs
         const int warps = POOL_THREADS / 32;
-        int gx = (4 * sms + BH - 1) / BH;
-        gx = max(1, min(gx, (r.n_past + warps - 1) / warps));
+        const int gx_max = max(1, occ * sms / BH);
+        const int per_warp = (r.n_past + warps * gx_max - 1) / (warps * gx_max);
+        const int gx = max(1, (r.n_past + warps * per_warp - 1) / (warps * per_warp));
         kern<<<dim3(gx, BH), POOL_THREADS, smem, st>>>(k, r.qbar, r);
         }
     }
