@@ -1,7 +1,7 @@
 """Benchmark of the Velox geometry-routed attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload headline|sweep|pipeline|robustness|rollout] [--P 48]
+                    [--workload headline|sweep|pipeline|robustness|rollout|overlap] [--P 48]
 
 One step = one pass of the whole hot path over one chunk's synthetic inputs,
 with the KV cache resident in HBM: frustum slices of every past chunk, slice
@@ -31,6 +31,10 @@ sparse and dense attention at each P.
 in --denoise-steps steps of --layers layers (pooled-key-cache routing and
 sparse attention over a KV cache sized for all of them), with the geometry
 built at each chunk boundary or pipelined one chunk ahead.
+
+--workload overlap times the slice-overlap kernel at the headline size and on a
+stress shape (64 scenes at 256 x 384 against 96 slices) against a measured
+float64 FMA rate.
 """
 from __future__ import annotations
 
@@ -919,6 +923,84 @@ def run_rollout(args):
         print(json.dumps(out), flush=True)
 
 
+# float64 operations of one overlap point test, from the method's formulas (a
+# division counts as one): per (point, slice) q = R p + t (9 mul + 9 add) and
+# u, v = f * (q_xy / q_z) + c (2 div + 2 mul + 2 add); per point, shared by the P
+# slices, the back-projection (2 sub + 2 div + 2 mul) and p_w = R^T (p_c - t)
+# (3 sub + 9 mul + 6 add).
+OVERLAP_FLOPS_PER_TEST = 24.0
+OVERLAP_FLOPS_PER_POINT = 24.0
+
+
+def run_overlap(args):
+    """The slice-overlap kernel at the headline size (latency-bound: us and
+    point tests per second) and on a stress shape where its float64 ALU work
+    dominates: 64 scenes at 256 x 384 (one frame per chunk) against 96 past
+    slices, 604 M point tests. Its rate is set against a measured float64 FMA
+    ceiling (velox_fp64_fma_bench)."""
+    import torch
+    from geometry_routed_block_b200 import velox as vx
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    reps = max(3, min(args.steps, 50))
+    # headline size
+    geo = synth.geometry_only(3)
+    s = synth.shape_for(3)
+    sl = vx.slices_build(dev(geo.past_depth[0]), dev(geo.past_poses[0]), dev(geo.past_intr[0]))
+    cd, cc = dev(geo.cur_depth), dev(geo.cur_cam)
+    counts = vx.block_overlap(cd, cc, sl[None], s.F, s.T)
+    for _ in range(3):
+        vx.block_overlap(cd, cc, sl[None], s.F, s.T, out=counts)
+    t_small = time_loop(torch, lambda: vx.block_overlap(cd, cc, sl[None], s.F, s.T, out=counts), reps)
+    tests_small = s.B * s.Nq * s.P
+    # float64 FMA ceiling
+    props = torch.cuda.get_device_properties(device)
+    fma_out = torch.zeros(1, dtype=torch.float64, device=device)
+    blocks, threads, iters = props.multi_processor_count * 8, 256, 1 << 14
+    fl = vx.fp64_fma_bench(fma_out, blocks, threads, iters)
+    t_fma = time_loop(torch, lambda: vx.fp64_fma_bench(fma_out, blocks, threads, iters), 5)
+    fp64_peak = fl / (t_fma * 1e-3) / 1e12
+    # stress shape
+    B, P, Hp, Wp, T = 64, 96, 256, 384, 128
+    g = synth.stress_geometry(B, P, Hp, Wp, seed=1010)
+    pd = dev(g["past_depth"].reshape(B * P, *g["past_depth"].shape[2:]))
+    slices = vx.slices_build(pd, dev(g["past_poses"].reshape(B * P, 12)),
+                             dev(g["past_intr"].reshape(B * P, 4))).view(B, P, 18)
+    cd, cc = dev(g["cur_depth"]), dev(g["cur_cam"])
+    counts = vx.block_overlap(cd, cc, slices, 1, T)
+    for _ in range(2):
+        vx.block_overlap(cd, cc, slices, 1, T, out=counts)
+    t_big = time_loop(torch, lambda: vx.block_overlap(cd, cc, slices, 1, T, out=counts), 10)
+    points = B * Hp * Wp
+    tests = points * P
+    flops = tests * OVERLAP_FLOPS_PER_TEST + points * OVERLAP_FLOPS_PER_POINT
+    achieved = flops / (t_big * 1e-3) / 1e12
+    covered = float((counts.sum(-1) > 0).float().mean().item())
+    out = {
+        "workload": "slice overlap (step 3 of the method's geometry): headline size and a stress shape",
+        "data": "synthetic", "n_gpus": 1,
+        "headline": {"shape": "B1, 3x32x48 tokens (T 128), 48 slices", "ms": round(t_small, 4),
+                     "point_tests": tests_small,
+                     "point_tests_per_s": round(tests_small / (t_small * 1e-3), 1),
+                     "note": "one launch, latency-bound; an HBM fraction is meaningless here"},
+        "stress": {"shape": f"B{B} scenes, {Hp}x{Wp} (1 frame per chunk, T {T}), {P} slices",
+                   "ms": round(t_big, 4), "point_tests": tests,
+                   "point_tests_per_s": round(tests / (t_big * 1e-3), 1),
+                   "fp64_flops_per_test": OVERLAP_FLOPS_PER_TEST,
+                   "achieved_fp64_tflops": round(achieved, 3),
+                   "covered_query_block_fraction": round(covered, 4)},
+        "roofline": {"bound": "alu", "achieved": round(achieved, 3), "peak": round(fp64_peak, 3),
+                     "unit": "TFLOP/s", "frac": round(achieved / fp64_peak, 4),
+                     "peak_kind": "measured float64 FMA rate (velox_fp64_fma_bench, FMA = 2 FLOP)",
+                     "traffic": None},
+    }
+    print(json.dumps(out), flush=True)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -962,7 +1044,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
     ap.add_argument("--workload", default="headline",
-                    choices=["headline", "sweep", "pipeline", "robustness", "rollout"])
+                    choices=["headline", "sweep", "pipeline", "robustness", "rollout", "overlap"])
     ap.add_argument("--chunks", type=int, default=4, help="chunks (rollout workload)")
     ap.add_argument("--denoise-steps", type=int, default=4, help="steps per chunk (rollout)")
     ap.add_argument("--layers", type=int, default=30, help="layers (pipeline workload)")
@@ -977,6 +1059,8 @@ def main():
         run_robustness(args)
     elif args.workload == "rollout":
         run_rollout(args)
+    elif args.workload == "overlap":
+        run_overlap(args)
     else:
         run_gpu(args)
 

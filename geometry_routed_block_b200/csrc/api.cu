@@ -217,6 +217,12 @@ int velox_depth_multiwarp(const float* past_depth, const velox_slice_t* past_cam
                                    ws, as_stream(stream));
 }
 
+int velox_fp64_fma_bench(double* out, int blocks, int threads, int iters, void* stream) {
+    if (!out || blocks < 1 || threads < 32 || threads > 1024 || (threads % 32) != 0 || iters < 1)
+        return VELOX_EINVAL;
+    return velox::fp64_fma_launch(out, blocks, threads, iters, as_stream(stream));
+}
+
 int velox_cast_bf16(const float* x, uint16_t* y, size_t n, void* stream) {
     if (!x || !y) return VELOX_EINVAL;
     if (n == 0) return VELOX_OK;

@@ -296,6 +296,31 @@ int multiwarp_launch(const float* past_depth, const velox_slice_t* past, const v
     return launch_status();
 }
 
+// float64 FMA throughput: 8 independent chains per thread (enough to cover the
+// pipe latency with a few warps per scheduler); a chain converges to
+// y / (1 - x), never to 0, so the store below never happens but the compiler
+// cannot drop the work.
+__global__ void fp64_fma_kernel(double* out, int iters) {
+    const double x = 0.999999, y = 1e-7 * (threadIdx.x + 1);
+    double a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = 1.0 + i + 1e-3 * threadIdx.x;
+#pragma unroll 4
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = fma(a[i], x, y);
+    }
+    double s = 0.0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s += a[i];
+    if (s == 0.0) out[0] = s;
+}
+
+int fp64_fma_launch(double* out, int blocks, int threads, int iters, cudaStream_t st) {
+    fp64_fma_kernel<<<blocks, threads, 0, st>>>(out, iters);
+    return launch_status();
+}
+
 int cast_bf16_launch(const float* x, uint16_t* y, size_t n, cudaStream_t st) {
     const size_t blocks = (n + 255) / 256;
     const int g = static_cast<int>(blocks < 148 * 16 ? (blocks ? blocks : 1) : 148 * 16);

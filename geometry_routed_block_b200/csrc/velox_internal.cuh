@@ -52,5 +52,6 @@ int kbar_append_launch(const void* k, int dtype, int BH, int Nk, int Nq, int d, 
                        int cap, float* kbar, cudaStream_t st);
 
 int cast_bf16_launch(const float* x, uint16_t* y, size_t n, cudaStream_t st);
+int fp64_fma_launch(double* out, int blocks, int threads, int iters, cudaStream_t st);
 
 }  // namespace velox

@@ -394,6 +394,35 @@ def _loop(cfg: int, seed: int, s: Shape, heads: tuple | None = None) -> Case:
                 meta={"view_overlap": ov, "heads": hsel})
 
 
+def stress_geometry(B: int, P: int, Hp: int, Wp: int, seed: int, fov_deg: float = 60.0,
+                    past_grid: tuple = (32, 48)) -> dict:
+    """B independent rooms (workload 3's scene generator, one seed per scene) seen
+    along workload 3's camera loop: the current chunk (index P) has a depth map at
+    Hp x Wp by ray cast; the P past chunks' depth maps are cast at the coarser
+    `past_grid` (they only fix each slice's [min, max]); every camera's intrinsics
+    are for the Hp x Wp grid. Returns float32 arrays cur_depth [B,Hp,Wp],
+    cur_cam [B,18], past_depth [B,P,h,w], past_poses [B,P,12], past_intr [B,P,4]."""
+    intr = intrinsics(Hp, Wp, fov_deg)
+    intr_lr = intrinsics(past_grid[0], past_grid[1], fov_deg)
+    poses = [loop_pose(n)[0] for n in range(P + 1)]
+    out = {"cur_depth": np.empty((B, Hp, Wp), np.float32),
+           "cur_cam": np.empty((B, CAM_FLOATS), np.float32),
+           "past_depth": np.empty((B, P) + tuple(past_grid), np.float32),
+           "past_poses": np.tile(np.stack(poses[:P]), (B, 1, 1)).astype(np.float32),
+           "past_intr": np.tile(intr, (B, P, 1)).astype(np.float32)}
+
+    def scene_job(b):
+        scene = room_scene(np.random.default_rng([seed, b]))
+        out["cur_depth"][b] = render_depth(scene, poses[P], intr, Hp, Wp)
+        out["cur_cam"][b] = camera_record(poses[P], intr)
+        for j in range(P):
+            out["past_depth"][b, j] = render_depth(scene, poses[j], intr_lr, *past_grid)
+
+    with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(scene_job, range(B)))
+    return out
+
+
 def perturb_depth(depth: np.ndarray, rng: np.random.Generator, noise_sd: float = 0.0,
                   hole_frac: float = 0.0, scale: float = 1.0) -> np.ndarray:
     """Depth-estimation error model for robustness studies (input generation,

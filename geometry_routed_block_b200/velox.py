@@ -51,6 +51,7 @@ SIGNATURES = {
     "velox_cast_bf16": (_c_int, [_vp, _vp, _c_size, _vp]),
     "velox_depth_multiwarp_noalloc": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_float,
                                                _vp, _vp]),
+    "velox_fp64_fma_bench": (_c_int, [_vp, _c_int, _c_int, _c_int, _vp]),
     "velox_kbar_cache_bytes": (_c_size, [_c_int] * 6),
     "velox_kbar_append": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                    _vp, _c_int, _vp]),
@@ -274,6 +275,14 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torc
                                      T, float(scale), _ptr(out), _ptr(lse), _ptr(status),
                                      _stream(stream)), "velox_sparse_attn_fwd")
     return out, lse
+
+
+def fp64_fma_bench(out: torch.Tensor, blocks: int, threads: int, iters: int, stream=None) -> int:
+    """Launches the float64 FMA throughput kernel; returns its FLOP count."""
+    _expect(out, torch.float64, "out")
+    _check(lib.velox_fp64_fma_bench(_ptr(out), int(blocks), int(threads), int(iters),
+                                    _stream(stream)), "velox_fp64_fma_bench")
+    return 16 * int(blocks) * int(threads) * int(iters)
 
 
 def cast_bf16(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

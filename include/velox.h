@@ -269,6 +269,17 @@ VELOX_API int velox_depth_multiwarp_noalloc(const float* past_depth,
  */
 VELOX_API int velox_cast_bf16(const float* x, uint16_t* y, size_t n, void* stream);
 
+/*
+ * Measurement helper, not a step of the method: blocks x threads threads each
+ * run `iters` rounds of 8 independent float64 fused multiply-adds (2 FLOP each:
+ * blocks * threads * iters * 16 FLOP per call), the ceiling that the float64
+ * geometry (velox_block_overlap) is compared with. `out` (one double, device)
+ * is written only in a case that does not occur, so the work cannot be
+ * optimised away. Errors: VELOX_EINVAL for NULL out, blocks < 1, threads not a
+ * multiple of 32 in [32, 1024], iters < 1.
+ */
+VELOX_API int velox_fp64_fma_bench(double* out, int blocks, int threads, int iters, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

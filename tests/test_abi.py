@@ -119,3 +119,12 @@ def test_geometry_rejects(lib):
     assert mw(FAKE, FAKE, FAKE, 4, 16, 16, 0.01, FAKE, FAKE, 8, NULL) == -1
     assert mw(FAKE, FAKE, FAKE, 0, 16, 16, 0.01, FAKE, FAKE, 1 << 20, NULL) == -1
     assert lib.velox_cast_bf16(NULL, FAKE, 4, NULL) == -1
+
+
+def test_fp64_fma_bench_rejects(lib):
+    f = lib.velox_fp64_fma_bench
+    assert f(NULL, 1, 32, 1, NULL) == -1
+    assert f(FAKE, 0, 32, 1, NULL) == -1
+    assert f(FAKE, 1, 48, 1, NULL) == -1
+    assert f(FAKE, 1, 2048, 1, NULL) == -1
+    assert f(FAKE, 1, 32, 0, NULL) == -1

@@ -312,6 +312,37 @@ def test_rollout_p224_largest_size_geometry_routing_attention(vx):
         assert np.abs(lse[b, h, sl_].cpu().numpy() - lse_ref).max() < 1e-3
 
 
+@pytest.mark.parametrize("n_past", [255, 256, 257, 512, 513, 1024, 1025, 2048, 2049, 4096, 4097])
+def test_selection_sizes_cover_every_kernel_variant(vx, n_past):
+    """One query block (T = d = 64, two heads, fp32 routing) against n_past past
+    blocks of one block per chunk: every selection variant (one CTA per row with
+    1 to 16 keys per thread, the radix selection beyond 4096), the modulation,
+    and k_past from 1 to n_past - 1."""
+    rng = np.random.default_rng(n_past)
+    T, d, B, H, m = 64, 64, 1, 2, 1
+    q = rng.standard_normal((B, H, m * T, d), dtype=np.float32)
+    k = rng.standard_normal((B, H, (n_past + m) * T, d), dtype=np.float32)
+    counts = rng.integers(0, T + 1, size=(B, m, n_past)).astype(np.int32)
+    counts[..., rng.random(n_past) < 0.3] = 0
+    for k_past in (1, n_past // 3, n_past - 1):
+        got = vx.route_topk(dev(q), dev(k), dev(counts), 2.0, k_past + m, T).cpu().numpy()
+        want, s_mod = vo.route_topk(q, k, counts, 2.0, k_past + m, T)
+        assert compare_selection(got, want, s_mod, m) <= 1, (n_past, k_past)
+
+
+def test_overlap_stress_grid_exact(vx):
+    """A 256 x 384 grid (768 query blocks of 128 one-frame tokens) against 96
+    slices: counts bit-exact against the oracle for both scenes."""
+    g = synth.stress_geometry(2, 96, 256, 384, seed=77)
+    B, P = 2, 96
+    sl = vo.slices_build(g["past_depth"].reshape(B * P, 32, 48), g["past_poses"].reshape(B * P, 12),
+                         g["past_intr"].reshape(B * P, 4)).reshape(B, P, 18)
+    got = vx.block_overlap(dev(g["cur_depth"]), dev(g["cur_cam"]), dev(sl), 1, 128).cpu().numpy()
+    want = vo.block_overlap(g["cur_depth"], g["cur_cam"], sl, 1, 128)
+    assert np.array_equal(got, want)
+    assert (want.sum(-1) > 0).mean() > 0.5
+
+
 def test_route_exact_ties_break_to_the_smaller_index(vx):
     # past chunks 0-2 are copies, and so are 3-5: their pooled scores tie exactly
     # (in fp32 on the device and in fp64 in the oracle), so the selection is
