@@ -6,7 +6,9 @@
 One step = one pass of the whole hot path over one chunk's synthetic inputs,
 with the KV cache resident in HBM: frustum slices of every past chunk, slice
 overlap counts, geometry-modulated top-k routing (pooling + scores + select)
-and block-sparse attention over the routed blocks. `value` is the whole-job
+and block-sparse attention over the routed blocks. The slices and counts are
+built on a side stream while the keys are pooled (only the selection waits
+for them), as the method builds its slices asynchronously to denoising. `value` is the whole-job
 throughput in TFLOP/s of attention work on the kept blocks
 (4 * B * H * m * topk * T^2 * d per step) divided by the step time. The dense
 attention over every block (the build's own dense baseline) is timed
@@ -239,16 +241,19 @@ class Workload:
         self.lse = torch.empty((s.B, s.H, s.Nq), dtype=torch.float32, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.launches_per_step = 6  # slices, overlap, pool_q, pool_score, select, attention
+        # the geometry runs on a side stream; only the selection waits for its counts
+        self.side = torch.cuda.Stream(device=device)
+        self.geo_ready = torch.cuda.Event()
 
     def geometry(self):
         vx, s = self.vx, self.s
         vx.slices_build(self.past_depth, self.past_poses, self.past_intr, out=self.slices)
         vx.block_overlap(self.cur_depth, self.cur_cam, self.slices[None], s.F, s.T, out=self.counts)
 
-    def route(self):
+    def route(self, ready=None):
         s = self.s
         self.vx.route_topk(self.q, self.k, self.counts, s.alpha, s.topk, s.T, ws=self.ws,
-                           out=self.idx)
+                           out=self.idx, counts_ready=ready)
 
     def attend(self):
         self.vx.sparse_attn_fwd(self.q, self.k, self.v, self.idx, self.s.T, out=self.o,
@@ -258,19 +263,28 @@ class Workload:
         self.vx.sparse_attn_fwd(self.q, self.k, self.v, None, self.s.T, out=self.o_dense,
                                 want_lse=False, status=self.status)
 
-    def step(self, ev=None):
-        if ev is None:
+    def step(self, ev=None, route=None):
+        """Slices and overlap counts on the side stream while the keys are pooled
+        on the current one (the selection waits for the counts through an
+        event), then attention. ev: events for geometry (ev0 -> ev1, side
+        stream), routing (ev0 -> ev2, including any wait for the counts) and
+        attention (ev2 -> ev3)."""
+        torch = self.torch
+        main = torch.cuda.current_stream()
+        self.side.wait_stream(main)  # this step's inputs were written on `main`
+        if ev is not None:
+            ev[0].record(main)
+        with torch.cuda.stream(self.side):
             self.geometry()
-            self.route()
-            self.attend()
-            return
-        ev[0].record()
-        self.geometry()
-        ev[1].record()
-        self.route()
-        ev[2].record()
+            if ev is not None:
+                ev[1].record(self.side)
+            self.geo_ready.record(self.side)
+        (route or self.route)(ready=self.geo_ready)
+        if ev is not None:
+            ev[2].record(main)
         self.attend()
-        ev[3].record()
+        if ev is not None:
+            ev[3].record(main)
 
 
 def reduce_max(values, device=None):
@@ -349,7 +363,7 @@ def run_gpu(args):
     clocks = clk.summary()
     ms_total = t_start.elapsed_time(t_end)
     geo_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    route_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    route_ms = statistics.mean(e[0].elapsed_time(e[2]) for e in evs)
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     status = int(w.status.item())
 
@@ -359,13 +373,12 @@ def run_gpu(args):
     append_ms = time_loop(torch, lambda: [w.vx.kbar_append(w.k, s.Nq, s.T, j, kbar)
                                           for j in range(s.P)], 3) / s.P
 
-    def route_cached():
-        w.vx.route_topk_cached(w.q, kbar, s.P, w.counts, s.alpha, s.topk, s.T, ws=w.ws, out=w.idx)
+    def route_cached(ready=None):
+        w.vx.route_topk_cached(w.q, kbar, s.P, w.counts, s.alpha, s.topk, s.T, ws=w.ws, out=w.idx,
+                               counts_ready=ready)
 
     def step_cached():
-        w.geometry()
-        route_cached()
-        w.attend()
+        w.step(route=route_cached)
 
     route_cached()
     route_cached_ms = time_loop(torch, route_cached, 20)
