@@ -147,9 +147,9 @@ VELOX_API size_t velox_route_topk_workspace_size(int B, int H, int Nq, int Nk, i
  *   topk - m past blocks with the largest s' are added (equal s': the smaller
  *   kb first). topk counts the current blocks.
  * Errors: VELOX_EINVAL for sizes that are not multiples (Nq % T, Nk % Nq),
- * topk < m or topk > Nk/T, ws_bytes too small, NULL or misaligned (16 B)
- * pointers; VELOX_EUNSUPPORTED for T not in {64,128}, d not in {64,128}, or an
- * unknown dtype.
+ * more than 8192 key blocks (Nk/T), topk < m or topk > Nk/T, ws_bytes too
+ * small, NULL or misaligned (16 B) pointers; VELOX_EUNSUPPORTED for T not in
+ * {64,128}, d not in {64,128}, or an unknown dtype.
  */
 VELOX_API int velox_route_topk(const void* q, const void* k, int dtype, int B, int H, int Nq, int Nk, int d,
                      int T, const int32_t* counts, float alpha, int topk, int32_t* idx, void* ws,
