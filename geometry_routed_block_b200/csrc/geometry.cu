@@ -71,10 +71,16 @@ __device__ __forceinline__ void to_camera(double xw, double yw, double zw, const
 }
 
 // continuous pixel coordinates u = fx*(qx/qz)+cx, v = fy*(qy/qz)+cy (qz > 0)
+__device__ __forceinline__ double image_u(double qx, double qz, const Cam64& k) {
+    return __dadd_rn(__dmul_rn(k.fx, __ddiv_rn(qx, qz)), k.cx);
+}
+__device__ __forceinline__ double image_v(double qy, double qz, const Cam64& k) {
+    return __dadd_rn(__dmul_rn(k.fy, __ddiv_rn(qy, qz)), k.cy);
+}
 __device__ __forceinline__ void image_coords(double qx, double qy, double qz, const Cam64& k,
                                              double& uu, double& vv) {
-    uu = __dadd_rn(__dmul_rn(k.fx, __ddiv_rn(qx, qz)), k.cx);
-    vv = __dadd_rn(__dmul_rn(k.fy, __ddiv_rn(qy, qz)), k.cy);
+    uu = image_u(qx, qz, k);
+    vv = image_v(qy, qz, k);
 }
 
 // ---------------------------------------------------------------- slices
@@ -127,13 +133,20 @@ __global__ void __launch_bounds__(256) slices_kernel(const float* __restrict__ d
 
 constexpr int CAMS_PER_CTA = 8;
 
-// grid (m, ceil(P / CAMS_PER_CTA), B), one thread per token of the query block
+// grid (m, ceil(P / CAMS_PER_CTA), B), one thread per token of the query block.
+// The CTA's slices are widened to float64 once, into shared memory; a point
+// whose horizontal coordinate is already off the grid skips the vertical one
+// (the same operations decide the count, only fewer of them run).
 __global__ void overlap_kernel(const float* __restrict__ depth, const velox_slice_t* __restrict__ cur,
                                const velox_slice_t* __restrict__ slices, int P, int Hp, int Wp,
                                int T, int m, int32_t* __restrict__ counts) {
+    __shared__ Cam64 cams_s[CAMS_PER_CTA];
     const int qb = blockIdx.x;
     const int b = blockIdx.z;
     const int j0 = blockIdx.y * CAMS_PER_CTA;
+    if (threadIdx.x < CAMS_PER_CTA && j0 + static_cast<int>(threadIdx.x) < P)
+        cams_s[threadIdx.x] = widen_cam(slices[static_cast<size_t>(b) * P + j0 + threadIdx.x]);
+    __syncthreads();
     const int HW = Hp * Wp;
     const int tau = qb * T + threadIdx.x;
     const int pix = tau % HW;
@@ -151,13 +164,15 @@ __global__ void overlap_kernel(const float* __restrict__ depth, const velox_slic
         if (j >= P) break;  // uniform across the CTA
         bool inside = false;
         if (valid) {
-            const Cam64 k = widen_cam(slices[static_cast<size_t>(b) * P + j]);
+            const Cam64& k = cams_s[jj];
             double qx, qy, qz;
             to_camera(xw, yw, zw, k, qx, qy, qz);
             if (qz > 0.0 && qz >= k.znear && qz <= k.zfar) {
-                double uu, vv;
-                image_coords(qx, qy, qz, k, uu, vv);
-                inside = uu >= 0.0 && uu < Wd && vv >= 0.0 && vv < Hd;
+                const double uu = image_u(qx, qz, k);
+                if (uu >= 0.0 && uu < Wd) {
+                    const double vv = image_v(qy, qz, k);
+                    inside = vv >= 0.0 && vv < Hd;
+                }
             }
         }
         const int cnt = __syncthreads_count(inside);
