@@ -448,8 +448,9 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_kernel(const SelArgs a)
 // the keys above u and the first equal ones in index order, at offsets from a
 // prefix over the warps' counts. Padding keys are 0, below every real key.
 constexpr int SEL_CTA_THREADS = 256;  // measured against 64 and 128
+constexpr bool SEL_RADIX = true;
 
-template <int THREADS, int CH>
+template <int THREADS, int CH, bool RADIX>
 __global__ void __launch_bounds__(THREADS) select_cta_kernel(const SelArgs a) {
     constexpr int SEL_CTA_WARPS = THREADS / 32;
     extern __shared__ uint32_t keys_s[];  // [n_past]
@@ -503,10 +504,68 @@ __global__ void __launch_bounds__(THREADS) select_cta_kernel(const SelArgs a) {
         kmin = min(kmin, span[0][w]);
         kmax = max(kmax, span[1][w]);
     }
+    uint32_t u;
+    if constexpr (RADIX) {
+        // 8-bit digits from the top: per round a 256-bin histogram of the digits
+        // of the keys that still match the chosen prefix (equal digits within a
+        // warp are added by one atomic), then warp 0 finds the digit that holds
+        // the remaining-th largest key by a scan from the top bin down
+        __shared__ int hist[256];
+        __shared__ int pick[2];
+        uint32_t prefix = 0, pmask = 0;
+        int remaining = k_past;
+#pragma unroll 1
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int i = t; i < 256; i += THREADS) hist[i] = 0;
+            __syncthreads();
+#pragma unroll
+            for (int c = 0; c < CH; ++c) {
+                const int i = c * THREADS + t;
+                const bool in = i < n_past && (key[c] & pmask) == prefix;
+                const int dg = in ? static_cast<int>((key[c] >> shift) & 255u) : -1;
+                const unsigned peers = __match_any_sync(FULL, dg);
+                if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[dg], __popc(peers));
+            }
+            __syncthreads();
+            if (warp == 0) {
+                int cnt[8], tot = 0;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    cnt[q] = hist[255 - 8 * lane - q];
+                    tot += cnt[q];
+                }
+                int incl = tot;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(FULL, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                const int excl = incl - tot;
+                if (excl < remaining && remaining <= incl) {  // exactly one lane
+                    int acc = excl;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (acc + cnt[q] >= remaining) {
+                            pick[0] = 255 - 8 * lane - q;
+                            pick[1] = acc;
+                            break;
+                        }
+                        acc += cnt[q];
+                    }
+                }
+            }
+            __syncthreads();
+            remaining -= pick[1];
+            prefix |= static_cast<uint32_t>(pick[0]) << shift;
+            pmask |= 0xFFu << shift;
+            __syncthreads();  // pick and hist are rewritten next round
+        }
+        u = prefix;
+    } else {
     // bits above the highest one where min and max differ are u's already
     const uint32_t diff = kmin ^ kmax;
     const int top = diff ? 31 - __clz(diff) : -1;
-    uint32_t u = top < 0 ? kmax : (kmax & ~((2u << top) - 1u));
+    u = top < 0 ? kmax : (kmax & ~((2u << top) - 1u));
 #pragma unroll 1
     for (int bit = top; bit >= 0; --bit) {
         const uint32_t cand = u | (1u << bit);
@@ -521,6 +580,7 @@ __global__ void __launch_bounds__(THREADS) select_cta_kernel(const SelArgs a) {
 #pragma unroll
         for (int w = 0; w < SEL_CTA_WARPS; ++w) tot += part[buf][w];
         if (tot >= k_past) u = cand;
+    }
     }
     // emission: warp w owns keys [s0, s1) of the row
     const unsigned lt = (1u << lane) - 1u;
@@ -569,15 +629,15 @@ int select_launch(const SelArgs& a, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(a.n_past) * sizeof(uint32_t);
     const dim3 grid(a.rows), block(TH);
     if (a.n_past <= TH * 1)
-        select_cta_kernel<TH, 1><<<grid, block, smem, st>>>(a);
+        select_cta_kernel<TH, 1, SEL_RADIX><<<grid, block, smem, st>>>(a);
     else if (a.n_past <= TH * 2)
-        select_cta_kernel<TH, 2><<<grid, block, smem, st>>>(a);
+        select_cta_kernel<TH, 2, SEL_RADIX><<<grid, block, smem, st>>>(a);
     else if (a.n_past <= TH * 4)
-        select_cta_kernel<TH, 4><<<grid, block, smem, st>>>(a);
+        select_cta_kernel<TH, 4, SEL_RADIX><<<grid, block, smem, st>>>(a);
     else if (a.n_past <= TH * 8)
-        select_cta_kernel<TH, 8><<<grid, block, smem, st>>>(a);
+        select_cta_kernel<TH, 8, SEL_RADIX><<<grid, block, smem, st>>>(a);
     else if (a.n_past <= TH * 16)
-        select_cta_kernel<TH, 16><<<grid, block, smem, st>>>(a);
+        select_cta_kernel<TH, 16, SEL_RADIX><<<grid, block, smem, st>>>(a);
     else
         select_kernel<<<(a.rows + SEL_WARPS - 1) / SEL_WARPS, SEL_WARPS * 32, 0, st>>>(a);
     return VELOX_OK;
