@@ -335,7 +335,8 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
 
     cfg = 4 if args.workload == "sweep" else 3
-    case = synth.make_case(cfg, seed=rank_seed(cfg, rank), P=args.P)
+    case = (synth.make_case(cfg, seed=rank_seed(cfg, rank), P=args.P, T=args.T, d=args.d)
+            if cfg == 4 else synth.make_case(cfg, seed=rank_seed(cfg, rank), P=args.P))
     s = case.shape
     w = Workload(case, device)
     peaks, peak_kind = load_peaks()
@@ -501,7 +502,8 @@ def run_gpu(args):
         },
         "roofline": {
             "bound": "tensor",
-            "kernel": "attn_pp_kernel (sparse walk, kept blocks)",
+            "kernel": ("attn_pp_kernel (sparse walk, kept blocks)" if (s.T, s.d) == (128, 128)
+                       else f"attn_fwd_kernel<d={s.d},T={s.T}> (sparse walk, kept blocks)"),
             "achieved": round(attn_tflops, 2),
             "peak": peak_t,
             "peak_kind": f"bf16 sustained ({peak_kind})",
@@ -1062,6 +1064,8 @@ def main():
     ap.add_argument("--denoise-steps", type=int, default=4, help="steps per chunk (rollout)")
     ap.add_argument("--layers", type=int, default=30, help="layers (pipeline workload)")
     ap.add_argument("--P", type=int, default=None, help="past chunks (sweep workload)")
+    ap.add_argument("--T", type=int, default=None, help="block size (sweep workload: 64 or 128)")
+    ap.add_argument("--d", type=int, default=None, help="head dim (sweep workload: 64 or 128)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":

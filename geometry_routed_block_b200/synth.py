@@ -80,11 +80,14 @@ SWEEP_P = (8, 16, 24, 32, 48, 96)
 
 
 def shape_for(cfg: int, P: int | None = None, H: int | None = None,
-              layers: int | None = None) -> Shape:
+              layers: int | None = None, T: int | None = None, d: int | None = None) -> Shape:
     if cfg == 4:
         base = SHAPES[3]
         P = 48 if P is None else P
-        s = Shape(**{**base.__dict__, "P": P, "topk": topk_for(P)})
+        T = base.T if T is None else T
+        d = base.d if d is None else d
+        m = base.F * base.Hp * base.Wp // T
+        s = Shape(**{**base.__dict__, "P": P, "T": T, "d": d, "topk": topk_for(P, m)})
     else:
         s = Shape(**SHAPES[cfg].__dict__)
         if P is not None and P != s.P:
@@ -439,12 +442,14 @@ def perturb_depth(depth: np.ndarray, rng: np.random.Generator, noise_sd: float =
 
 
 def make_case(cfg: int, seed: int | None = None, P: int | None = None, H: int | None = None,
-              layers: int | None = None, heads: tuple | None = None) -> Case:
-    """Build workload `cfg` (1..5). Default seed is 1000 + cfg."""
+              layers: int | None = None, heads: tuple | None = None, T: int | None = None,
+              d: int | None = None) -> Case:
+    """Build workload `cfg` (1..5). Default seed is 1000 + cfg. Workload 4 also
+    takes another block size T or head dim d."""
     seed = 1000 + cfg if seed is None else seed
     if cfg == 1:
         return _tiny(seed)
-    s = shape_for(cfg, P=P, H=H, layers=layers)
+    s = shape_for(cfg, P=P, H=H, layers=layers, T=T, d=d)
     if cfg == 2:
         return _walk(seed, s)
     return _loop(cfg, seed, s, heads=heads)
