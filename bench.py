@@ -60,9 +60,9 @@ METRIC = "chunk-48 routed attention ms & TFLOP/s (kept blocks), speedup vs dense
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM bytes of one sparse attention launch at this workload, from the ncu capture
-# summarised in profiles/attn_pp_kernel_chunk48_dram.md; reported only while the
-# kernel sources still hash to what was captured.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one sparse attention
+# launch at the headline workload, from a one-pass ncu capture of this kernel at full
+# size; reported only while the kernel sources still hash to what was captured.
 ATTN_TRAFFIC = {
     "bytes_per_launch": 642.18e6 + 22.82e6,
     "sources": {"attention_pp.cu": "13e4340e74204946", "attn_common.cuh": "edbf6bcdb3a2cde6",

@@ -20,8 +20,7 @@ no formula, constant or kernel):
        context selection over a KV cache that grows per chunk) and "심층 분석"
        (same four steps; the kernel really skips unneeded blocks).
 
-Where the pages are silent the oracle takes the plainest reading (all listed in
-DESIGN.md under "Readings"):
+Where the pages are silent the oracle takes the plainest reading:
   * modulation: s' = s + alpha * overlap on covered query blocks, overlap =
     count / T, covered = at least one point of the block inside some past slice;
   * block importance s = mean-pooled Q block . mean-pooled K block / sqrt(d),
