@@ -1,5 +1,5 @@
 """The benchmark's JSON line for the reference arm (the fp64 oracle on the host
-cores) runs on the CPU: its keys follow the contract the driver reads."""
+cores) runs on the CPU: it prints one line with the benchmark's documented keys."""
 import json
 import os
 import subprocess
