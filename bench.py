@@ -11,7 +11,7 @@ built on a side stream while the keys are pooled (only the selection waits
 for them), as the method builds its slices asynchronously to denoising. `value` is the whole-job
 throughput in TFLOP/s of attention work on the kept blocks
 (4 * B * H * m * topk * T^2 * d per step) divided by the step time. The dense
-attention over every block (the build's own dense baseline) is timed
+attention over every block (this library's own dense attention) is timed
 separately for the speedup.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own chunk
