@@ -16,7 +16,9 @@ separately for the speedup.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own chunk
 (seed + rank) -- heads/chunks are independent units, there is no data-path
-collective -- and the time is the max over ranks ("scaling": "weak").
+collective -- and the time is the max over ranks ("scaling": "weak"). With
+--shard heads the ranks split the heads of one chunk instead, replicate the
+geometry and all-gather O every step ("scaling": "strong").
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload (the oracle stands in for a reference
@@ -244,6 +246,7 @@ class Workload:
         # the geometry runs on a side stream; only the selection waits for its counts
         self.side = torch.cuda.Stream(device=device)
         self.geo_ready = torch.cuda.Event()
+        self.after_attend = None  # e.g. the all-gather of O when heads are sharded
 
     def geometry(self):
         vx, s = self.vx, self.s
@@ -258,6 +261,8 @@ class Workload:
     def attend(self):
         self.vx.sparse_attn_fwd(self.q, self.k, self.v, self.idx, self.s.T, out=self.o,
                                 lse=self.lse, status=self.status)
+        if self.after_attend is not None:
+            self.after_attend()
 
     def dense(self):
         self.vx.sparse_attn_fwd(self.q, self.k, self.v, None, self.s.T, out=self.o_dense,
@@ -302,6 +307,26 @@ def job_throughput(world: int, units_per_rank: float, ms: float) -> float:
     return world * units_per_rank / (ms * 1e-3)
 
 
+def head_range(H: int, world: int, rank: int) -> tuple:
+    """Heads [h0, h1) of `rank` when the H heads are split evenly over `world` ranks."""
+    if H % world:
+        raise ValueError(f"{H} heads do not split evenly over {world} ranks")
+    n = H // world
+    return rank * n, (rank + 1) * n
+
+
+def gather_heads(o_local, world: int):
+    """Every rank's [B, H/world, N, d] output -> the whole [B, H, N, d] on every rank
+    (heads rank-major, as head_range splits them): one all-gather."""
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return o_local
+    parts = [torch.empty_like(o_local) for _ in range(world)]
+    dist.all_gather(parts, o_local.contiguous())
+    return torch.cat(parts, dim=1)
+
+
 def rank_seed(cfg: int, rank: int) -> int:
     """Each rank runs its own chunk: the workload's seed offset by the rank."""
     return 1000 + cfg + rank
@@ -335,10 +360,19 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
 
     cfg = 4 if args.workload == "sweep" else 3
-    case = (synth.make_case(cfg, seed=rank_seed(cfg, rank), P=args.P, T=args.T, d=args.d)
-            if cfg == 4 else synth.make_case(cfg, seed=rank_seed(cfg, rank), P=args.P))
+    by_heads = args.shard == "heads"
+    extra = {"T": args.T, "d": args.d} if cfg == 4 else {}
+    if by_heads:
+        # one chunk for the whole job; each rank routes and attends its share of the
+        # heads (geometry replicated) and the heads' outputs are all-gathered
+        h0, h1 = head_range(synth.shape_for(cfg, P=args.P, **extra).H, world, rank)
+        case = synth.make_case(cfg, seed=1000 + cfg, P=args.P, heads=tuple(range(h0, h1)), **extra)
+    else:
+        case = synth.make_case(cfg, seed=rank_seed(cfg, rank), P=args.P, **extra)
     s = case.shape
     w = Workload(case, device)
+    if by_heads and world > 1:
+        w.after_attend = lambda: gather_heads(w.o, world)
     peaks, peak_kind = load_peaks()
 
     # warm-up (also the first-call costs: tensor-map encode, attribute set)
@@ -457,10 +491,12 @@ def run_gpu(args):
     ms_total, e2e_ms = reduce_max([ms_total, e2e_ms], device)
     ms_step = ms_total / args.steps
 
-    kf, df = kept_flops(s), dense_flops(s)
+    # per-rank work: the whole chunk, or this rank's share of the heads
+    share = world if by_heads else 1
+    kf, df = kept_flops(s) / share, dense_flops(s) / share
     value = job_throughput(world, kf, ms_step) / 1e12
     attn_tflops = kf / (attn_ms * 1e-3) / 1e12
-    rbytes = routing_bytes(s)
+    rbytes = routing_bytes(s) / share
     route_gbs = rbytes / (route_ms * 1e-3) / 1e9
     peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     out = {
@@ -472,7 +508,7 @@ def run_gpu(args):
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if by_heads else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
@@ -480,7 +516,9 @@ def run_gpu(args):
             "workload": workload_desc(s),
             "l2": "inputs larger than L2 (past K and V are 1.39 GB each at chunk 48); no flush",
             "kept_fraction": round(s.topk / s.nKB, 4),
-            "parallelism": f"replicated chunks x{world} (one per GPU, no collective)",
+            "parallelism": (f"heads split over {world} GPU(s), geometry replicated, O all-gathered "
+                            "each step" if by_heads
+                            else f"replicated chunks x{world} (one per GPU, no collective)"),
         },
         "routed_attn_ms": round(attn_ms, 4),
         "routing_ms": round(route_ms, 4),
@@ -510,7 +548,7 @@ def run_gpu(args):
             "unit": "TFLOP/s",
             "frac": round(attn_tflops / peak_t, 4),
             "frac_of_burst": round(attn_tflops / peaks["bf16_tflops"], 4),
-            "traffic": attn_traffic() if s.P == 48 and cfg == 3 else None,
+            "traffic": attn_traffic() if s.P == 48 and cfg == 3 and share == 1 else None,
         },
         "routing_roofline": {
             "bound": "hbm", "achieved": round(route_gbs, 1), "peak": peaks["hbm_gbs"],
@@ -1067,6 +1105,9 @@ def main():
     ap.add_argument("--T", type=int, default=None, help="block size (sweep workload: 64 or 128)")
     ap.add_argument("--d", type=int, default=None, help="head dim (sweep workload: 64 or 128)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="chunks", choices=["chunks", "heads"],
+                    help="multi-GPU: one chunk per GPU (weak scaling) or the heads of one "
+                         "chunk split over the GPUs with an all-gather of O (strong scaling)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

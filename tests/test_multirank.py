@@ -52,3 +52,38 @@ def test_single_process_is_identity():
     import bench
     assert bench.reduce_max([1.5, 2.5]) == [1.5, 2.5]
     assert bench.job_throughput(1, 1e12, 1.0) == pytest.approx(1e15)
+
+
+def _heads_main(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    import bench
+    B, H, N, d = 2, 24, 8, 4
+    full = torch.arange(B * H * N * d, dtype=torch.float32).view(B, H, N, d)
+    h0, h1 = bench.head_range(H, world, rank)
+    got = bench.gather_heads(full[:, h0:h1].clone(), world)
+    out[rank] = ((h0, h1), bool(torch.equal(got, full)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_heads_split_and_gather_over_two_gloo_ranks():
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_heads_main, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0] == ((0, 12), True) and res[1] == ((12, 24), True)
+
+
+def test_head_range_rejects_uneven_splits():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert [bench.head_range(24, 8, r) for r in (0, 7)] == [(0, 3), (21, 24)]
+    with pytest.raises(ValueError):
+        bench.head_range(24, 5, 0)
