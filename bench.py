@@ -422,6 +422,15 @@ def run_gpu(args):
     # ---- dense baseline, timed alone (inputs > L2, so no flush is needed)
     dense_reps = max(3, min(20, args.steps // 10))
     dense_ms = time_loop(torch, w.dense, dense_reps)
+    # context only, not on the path: PyTorch's own dense attention on the same tensors
+    sdpa_ms = None
+    try:
+        import torch.nn.functional as F
+        sdpa = lambda: F.scaled_dot_product_attention(w.q, w.k, w.v)
+        sdpa()
+        sdpa_ms = time_loop(torch, sdpa, dense_reps)
+    except RuntimeError:
+        pass
 
     # ---- end to end through the public API with host buffers: each step copies
     # the chunk's new inputs (Q, the current chunk's K and V, its depth map and
@@ -530,6 +539,12 @@ def run_gpu(args):
         "routing_hbm_frac": round(route_gbs / peaks["hbm_gbs"], 4),
         "speedup_vs_dense": round(dense_ms / (route_ms + attn_ms), 3),
         "attn_speedup_vs_dense": round(dense_ms / attn_ms, 3),
+        "torch_sdpa_dense": (None if sdpa_ms is None else
+                             {"ms": round(sdpa_ms, 4),
+                              "tflops": round(df / (sdpa_ms * 1e-3) / 1e12, 2),
+                              "routed_step_speedup": round(sdpa_ms / (route_ms + attn_ms), 3),
+                              "note": "torch.nn.functional.scaled_dot_product_attention on the "
+                                      "same tensors, every key block: context only"}),
         "allowed_speedup": round(s.nKB / s.topk, 3),
         "pooled_key_cache": {
             "append_ms_per_chunk": round(append_ms, 4),
