@@ -343,6 +343,35 @@ def test_overlap_stress_grid_exact(vx):
     assert (want.sum(-1) > 0).mean() > 0.5
 
 
+def test_overlap_exact_on_slice_boundaries(vx):
+    """Points that land on a slice's bounds up to float64 rounding: past cameras
+    with the current pose, depth intervals whose ends are depths of the map, and
+    principal points shifted by half a pixel so that pixel centres project onto
+    u = 0, u = W, v = 0 or v = H. The kernel's float32 shortcut must leave all
+    of these to the float64 test; counts match the oracle exactly."""
+    rng = np.random.default_rng(5)
+    Hp, Wp, T, F = 16, 24, 64, 1
+    pose = synth.pose_looking((0.3, 1.2, -0.7), (0.2, -0.1, 1.0))
+    intr = synth.intrinsics(Hp, Wp, 60.0)
+    depth = rng.uniform(1.0, 9.0, (1, Hp, Wp)).astype(np.float32)
+    depth[0, 3, 5] = np.float32(2.0)
+    depth[0, 7, 9] = np.float32(6.5)
+    cur = synth.camera_record(pose, intr)[None]
+    z = depth[0].ravel()
+    cams = []
+    for zn, zf in ((2.0, 6.5), (float(np.sort(z)[10]), float(np.sort(z)[-10])), (0.0, 100.0)):
+        for dcx, dcy in ((0.0, 0.0), (-0.5, 0.0), (0.5, 0.0), (0.0, -0.5), (0.0, 0.5)):
+            k = intr.copy()
+            k[2] += dcx
+            k[3] += dcy
+            cams.append(synth.camera_record(pose, k, zn, zf))
+    sl = np.stack(cams)[None]
+    got = vx.block_overlap(dev(depth), dev(cur), dev(sl), F, T).cpu().numpy()
+    want = vo.block_overlap(depth, cur, sl, F, T)
+    assert np.array_equal(got, want)
+    assert 0 < want.sum() < want.size * T
+
+
 def test_route_exact_ties_break_to_the_smaller_index(vx):
     # past chunks 0-2 are copies, and so are 3-5: their pooled scores tie exactly
     # (in fp32 on the device and in fp64 in the oracle), so the selection is
