@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(THREADS) select_cta_kernel(const SelArgs a) {
         // of the keys that still match the chosen prefix (equal digits within a
         // warp are added by one atomic), then warp 0 finds the digit that holds
         // the remaining-th largest key by a scan from the top bin down
-        __shared__ int hist[256];
+        __shared__ __align__(16) int hist[256];
         __shared__ int pick[2];
         uint32_t prefix = 0, pmask = 0;
         int remaining = k_past;
@@ -528,12 +528,13 @@ __global__ void __launch_bounds__(THREADS) select_cta_kernel(const SelArgs a) {
             }
             __syncthreads();
             if (warp == 0) {
-                int cnt[8], tot = 0;
+                // lane L takes bins 255-8L down to 248-8L: 32 contiguous bytes
+                const int4 lo = reinterpret_cast<const int4*>(hist)[62 - 2 * lane];
+                const int4 hi = reinterpret_cast<const int4*>(hist)[63 - 2 * lane];
+                const int cnt[8] = {hi.w, hi.z, hi.y, hi.x, lo.w, lo.z, lo.y, lo.x};
+                int tot = 0;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    cnt[q] = hist[255 - 8 * lane - q];
-                    tot += cnt[q];
-                }
+                for (int q = 0; q < 8; ++q) tot += cnt[q];
                 int incl = tot;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
