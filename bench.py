@@ -182,32 +182,94 @@ def cpu_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(case, head: int = 0, n_rows: int | None = None):
-    """Runs the oracle on: all geometry (slices + overlap counts), the routing
-    of one (batch, head) pair and the attention of `n_rows` query blocks of
-    that pair (all of them by default). Returns (estimated whole-step seconds,
-    sample seconds, description); the estimate scales the per-head routing by
-    B*H and the per-row attention by B*H*m."""
+SAMPLE_ROWS = 4  # query blocks of the sampled head whose attention the oracle computes
+
+
+def oracle_sample(case, head: int = 0, n_rows: int = SAMPLE_ROWS) -> dict:
+    """Runs the oracle on one bounded sample of a step: all geometry (slices +
+    overlap counts), the routing of one (batch, head) pair and the attention
+    of `n_rows` evenly spaced query blocks of that pair. Returns the measured
+    seconds of each part, the whole step extrapolated from them (geometry +
+    B*H routings + B*H*m query blocks at the sampled per-block time), and the
+    sample's counts and selection (for the parity check of the GPU's)."""
     from oracle import velox_oracle as vo
     s = case.shape
-    n_rows = s.m if n_rows is None else max(1, min(s.m, n_rows))
+    n_rows = max(1, min(s.m, n_rows))
     t0 = time.perf_counter()
     sl = vo.slices_build(case.past_depth[0], case.past_poses[0], case.past_intr[0])
     counts = vo.block_overlap(case.cur_depth, case.cur_cam, sl[None], s.F, s.T)
     t1 = time.perf_counter()
     q, k, v = case.q[0][:, head:head + 1], case.k[0][:, head:head + 1], case.v[0][:, head:head + 1]
-    idx, _ = vo.route_topk(q, k, counts, s.alpha, s.topk, s.T)
+    idx, s_mod = vo.route_topk(q, k, counts, s.alpha, s.topk, s.T)
     t2 = time.perf_counter()
-    step = max(1, s.m // n_rows)
-    rows = [(0, 0, qb) for qb in range(0, s.m, step)][:n_rows]
-    vo.sparse_attention(q, k, v, idx, s.T, rows=rows)
+    qbs = [int(round(i * (s.m - 1) / max(1, n_rows - 1))) for i in range(n_rows)]
+    vo.sparse_attention(q, k, v, idx, s.T, rows=[(0, 0, qb) for qb in qbs])
     t3 = time.perf_counter()
     pairs = s.B * s.H
-    est = (t1 - t0) + pairs * (t2 - t1) + pairs * s.m * (t3 - t2) / len(rows)
-    desc = (f"oracle (numpy fp64): all geometry, routing of 1 of {pairs} (batch, head) pairs and "
-            f"attention of {len(rows)} of its {s.m} query blocks; step time = geometry + "
+    per_row = (t3 - t2) / len(qbs)
+    est = (t1 - t0) + pairs * (t2 - t1) + pairs * s.m * per_row
+    desc = (f"oracle (numpy fp64) on a bounded sample of one step: all geometry (slices + "
+            f"overlap counts), routing of (batch 0, head {head}) and attention of {len(qbs)} of "
+            f"its {s.m} query blocks (qb {qbs}); the whole step is extrapolated as geometry + "
             f"{pairs} x routing + {pairs * s.m} x per-block attention")
-    return est, t3 - t0, desc
+    return {"geometry_s": t1 - t0, "routing_s_per_head": t2 - t1,
+            "attention_s_per_query_block": per_row, "sample_s": t3 - t0, "est_step_s": est,
+            "desc": desc, "counts": counts, "idx": idx, "s_mod": s_mod}
+
+
+def oracle_repeated(case, min_seconds: float, max_repeats: int = 64) -> dict:
+    """oracle_sample run again and again until `min_seconds` of host time have
+    gone by (at least once); every timing is the mean over the repeats."""
+    runs = [oracle_sample(case)]
+    t = runs[0]["sample_s"]
+    while t < min_seconds and len(runs) < max_repeats:
+        runs.append(oracle_sample(case))
+        t += runs[-1]["sample_s"]
+    r = dict(runs[0])
+    for key in ("geometry_s", "routing_s_per_head", "attention_s_per_query_block", "sample_s",
+                "est_step_s"):
+        r[key] = statistics.mean(x[key] for x in runs)
+    r["repeats"] = len(runs)
+    return r
+
+
+def oracle_single_thread(case, min_seconds: float = 2.0) -> dict:
+    """oracle_repeated with the BLAS thread pool limited to one thread."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        return oracle_repeated(case, min_seconds)
+
+
+def baseline_record(kf: float, r: dict, r1: dict | None) -> dict:
+    """The cpu_baseline object: the oracle's whole-step throughput extrapolated
+    from the sample `r` (all host threads) and, when given, `r1` (one thread)."""
+    out = {"value": round(kf / r["est_step_s"] / 1e12, 6), "unit": "TFLOP/s",
+           "cores": cpu_threads(), "kind": "oracle", "sample": r["desc"], "extrapolated": True,
+           "sample_seconds": round(r["sample_s"], 3), "repeats": r.get("repeats", 1),
+           "est_step_seconds": round(r["est_step_s"], 2),
+           "geometry_s": round(r["geometry_s"], 4),
+           "routing_s_per_head": round(r["routing_s_per_head"], 4),
+           "attention_s_per_query_block": round(r["attention_s_per_query_block"], 4)}
+    if r1 is not None:
+        out["single_thread"] = {
+            "value": round(kf / r1["est_step_s"] / 1e12, 6), "cores": 1,
+            "sample_seconds": round(r1["sample_s"], 3), "repeats": r1.get("repeats", 1),
+            "est_step_seconds": round(r1["est_step_s"], 2),
+            "routing_s_per_head": round(r1["routing_s_per_head"], 4),
+            "attention_s_per_query_block": round(r1["attention_s_per_query_block"], 4)}
+    return out
+
+
+def selection_ties(gpu_idx, oracle_idx, s_mod, m) -> dict:
+    """GPU selection vs the oracle's on the same rows under the parity rule
+    (equal, or differing only at blocks within 1e-4 of the threshold)."""
+    from tests.parity_utils import TIE_TOL, compare_selection
+    try:
+        ties = compare_selection(gpu_idx, oracle_idx, s_mod, m)
+        return {"rows": int(np.prod(gpu_idx.shape[:-1])), "near_tie_rows": ties,
+                "tie_tol": TIE_TOL, "ok": True}
+    except AssertionError as e:
+        return {"rows": int(np.prod(gpu_idx.shape[:-1])), "ok": False, "error": str(e)[:200]}
 
 
 # ----------------------------------------------------------------------------
@@ -230,17 +292,18 @@ class Workload:
             return torch.from_numpy(np.ascontiguousarray(a)).to(device)
 
         self.q, self.k, self.v = dev(case.q[0]), dev(case.k[0]), dev(case.v[0])
+        H = self.q.shape[1]  # the heads this process holds (all, or its share)
         self.past_depth = dev(case.past_depth[0])
         self.past_poses = dev(case.past_poses[0])
         self.past_intr = dev(case.past_intr[0])
         self.cur_depth, self.cur_cam = dev(case.cur_depth), dev(case.cur_cam)
         self.slices = torch.empty((s.P, 18), dtype=torch.float32, device=device)
         self.counts = torch.empty((s.B, s.m, s.P), dtype=torch.int32, device=device)
-        self.ws = vx.route_workspace(s.B, s.H, s.Nq, s.Nk, s.d, s.T, device)
-        self.idx = torch.empty((s.B, s.H, s.m, s.topk), dtype=torch.int32, device=device)
+        self.ws = vx.route_workspace(s.B, H, s.Nq, s.Nk, s.d, s.T, device)
+        self.idx = torch.empty((s.B, H, s.m, s.topk), dtype=torch.int32, device=device)
         self.o = torch.empty_like(self.q)
         self.o_dense = torch.empty_like(self.q)
-        self.lse = torch.empty((s.B, s.H, s.Nq), dtype=torch.float32, device=device)
+        self.lse = torch.empty((s.B, H, s.Nq), dtype=torch.float32, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.launches_per_step = 6  # slices, overlap, pool_q, pool_score, select, attention
         # the geometry runs on a side stream; only the selection waits for its counts
@@ -315,16 +378,21 @@ def head_range(H: int, world: int, rank: int) -> tuple:
     return rank * n, (rank + 1) * n
 
 
-def gather_heads(o_local, world: int):
-    """Every rank's [B, H/world, N, d] output -> the whole [B, H, N, d] on every rank
-    (heads rank-major, as head_range splits them): one all-gather."""
-    import torch
+def gather_heads(o_all, o_local, world: int):
+    """Every rank's [B, H/world, N, d] output o_local -> o_all [world * B, H/world, N, d]
+    (rank r's share at rows r*B .. r*B+B-1) on every rank, by one all-gather into
+    the preallocated buffer: in place when o_local is this rank's slice of
+    o_all. Returns the whole output as [B, H, N, d], heads in order (rank-major,
+    as head_range splits them): a view of o_all when B = 1, a permuted copy
+    otherwise."""
     import torch.distributed as dist
-    if world == 1:
-        return o_local
-    parts = [torch.empty_like(o_local) for _ in range(world)]
-    dist.all_gather(parts, o_local.contiguous())
-    return torch.cat(parts, dim=1)
+    if world > 1:
+        dist.all_gather_into_tensor(o_all, o_local)
+    WB, h, N, d = o_all.shape
+    B = WB // world
+    if B == 1:
+        return o_all.view(1, world * h, N, d)
+    return o_all.view(world, B, h, N, d).permute(1, 0, 2, 3, 4).reshape(B, world * h, N, d)
 
 
 def rank_seed(cfg: int, rank: int) -> int:
@@ -344,9 +412,59 @@ def time_loop(torch, fn, reps):
     return a.elapsed_time(b) / reps
 
 
+SWEEP_P = (8, 16, 24, 32, 96)
+
+
+def sweep_point(torch, vx, device, P: int, reps: int, peaks: dict, status):
+    """Workload 4 at P past chunks on this GPU (geometry from the synthetic
+    trajectory, Q/K/V drawn on the device with workload 3's structure): routing,
+    sparse attention and dense attention timed alone with CUDA events. Returns
+    the record and, for the oracle check, head 0's inputs and selection."""
+    geo = synth.geometry_only(4, P=P)
+    s = synth.shape_for(4, P=P)
+    q, k, v = draw_qkv_on_device(torch, s, geo.meta["view_overlap"], 1004 + P, device)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    slices = vx.slices_build(dev(geo.past_depth[0]), dev(geo.past_poses[0]), dev(geo.past_intr[0]))
+    counts = vx.block_overlap(dev(geo.cur_depth), dev(geo.cur_cam), slices[None], s.F, s.T)
+    ws = vx.route_workspace(s.B, s.H, s.Nq, s.Nk, s.d, s.T, device)
+    idx = torch.empty((s.B, s.H, s.m, s.topk), dtype=torch.int32, device=device)
+    o, o2 = torch.empty_like(q), torch.empty_like(q)
+    lse = torch.empty((s.B, s.H, s.Nq), dtype=torch.float32, device=device)
+    route = lambda: vx.route_topk(q, k, counts, s.alpha, s.topk, s.T, ws=ws, out=idx)
+    attend = lambda: vx.sparse_attn_fwd(q, k, v, idx, s.T, out=o, lse=lse, status=status)
+    dense = lambda: vx.sparse_attn_fwd(q, k, v, None, s.T, out=o2, want_lse=False, status=status)
+    for _ in range(3):
+        route()
+        attend()
+    dense()
+    t_route = time_loop(torch, route, reps)
+    t_attn = time_loop(torch, attend, reps)
+    t_dense = time_loop(torch, dense, max(2, reps // 4))
+    rbytes = routing_bytes(s)
+    kf, df = kept_flops(s), dense_flops(s)
+    attn_tf = kf / (t_attn * 1e-3) / 1e12
+    route_gbs = rbytes / (t_route * 1e-3) / 1e9
+    rec = {
+        "P": P, "key_blocks": s.nKB, "topk": s.topk, "kept_fraction": round(s.topk / s.nKB, 4),
+        "routing_ms": round(t_route, 4), "routing_gbs": round(route_gbs, 1),
+        "routing_hbm_frac": round(route_gbs / peaks["hbm_gbs"], 4),
+        "sparse_attn_ms": round(t_attn, 4), "attn_tflops_kept": round(attn_tf, 1),
+        "attn_tensor_frac": round(attn_tf / peaks["bf16_tflops"], 4),
+        "dense_attn_ms": round(t_dense, 4),
+        "dense_tflops": round(df / (t_dense * 1e-3) / 1e12, 1),
+        "speedup_vs_dense": round(t_dense / (t_route + t_attn), 3),
+        "attn_speedup_vs_dense": round(t_dense / t_attn, 3),
+        "allowed_speedup": round(s.nKB / s.topk, 3),
+    }
+    check = {"q": q[:, :1].cpu(), "k": k[:, :1].cpu(), "idx": idx[:, :1].cpu().numpy(),
+             "counts": counts.cpu().numpy(), "shape": s}
+    return rec, check
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
+    from geometry_routed_block_b200 import velox as vx
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -366,13 +484,19 @@ def run_gpu(args):
         # one chunk for the whole job; each rank routes and attends its share of the
         # heads (geometry replicated) and the heads' outputs are all-gathered
         h0, h1 = head_range(synth.shape_for(cfg, P=args.P, **extra).H, world, rank)
-        case = synth.make_case(cfg, seed=1000 + cfg, P=args.P, heads=tuple(range(h0, h1)), **extra)
+        heads = None if (h0, h1) == (0, synth.shape_for(cfg, P=args.P, **extra).H) else tuple(range(h0, h1))
+        case = synth.make_case(cfg, seed=1000 + cfg, P=args.P, heads=heads, **extra)
     else:
         case = synth.make_case(cfg, seed=rank_seed(cfg, rank), P=args.P, **extra)
     s = case.shape
     w = Workload(case, device)
+    o_all = None
     if by_heads and world > 1:
-        w.after_attend = lambda: gather_heads(w.o, world)
+        # this rank's heads are written straight into its slice of the gathered output
+        B_ = w.o.shape[0]
+        o_all = torch.empty((world * B_,) + tuple(w.o.shape[1:]), dtype=w.o.dtype, device=device)
+        w.o = o_all[rank * B_:(rank + 1) * B_]
+        w.after_attend = lambda: gather_heads(o_all, w.o, world)
     peaks, peak_kind = load_peaks()
 
     # warm-up (also the first-call costs: tensor-map encode, attribute set)
@@ -401,10 +525,11 @@ def run_gpu(args):
     route_ms = statistics.mean(e[0].elapsed_time(e[2]) for e in evs)
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     status = int(w.status.item())
+    gpu_idx = w.idx.cpu().numpy()
 
     # ---- pooled-key cache: each past chunk's key blocks pooled once when the chunk
     # was appended; per step the routing reads the 21 MB cache instead of 1.36 GB of K
-    kbar = w.vx.kbar_cache(s.B, s.H, s.P, s.Nq, s.d, s.T, device)
+    kbar = w.vx.kbar_cache(s.B, w.q.shape[1], s.P, s.Nq, s.d, s.T, device)
     append_ms = time_loop(torch, lambda: [w.vx.kbar_append(w.k, s.Nq, s.T, j, kbar)
                                           for j in range(s.P)], 3) / s.P
 
@@ -496,6 +621,24 @@ def run_gpu(args):
     e2e_ms = time_loop(torch, lambda: e2e_run(e2e_reps), 1) / e2e_reps
     h_o_ok = bool(torch.equal(h_o, w.o.cpu()))
 
+    # the host links alone: one step's uploads, its download, and both at once
+    def copies(up_on=True, down_on=True):
+        if up_on:
+            with torch.cuda.stream(up):
+                for key, h in (("q", h_q), ("k", h_k), ("v", h_v), ("depth", h_depth),
+                               ("cam", h_cam)):
+                    stage[0][key].copy_(h, non_blocking=True)
+        if down_on:
+            with torch.cuda.stream(down):
+                h_o.copy_(stage[1]["o"], non_blocking=True)
+        compute.wait_stream(up)
+        compute.wait_stream(down)
+
+    copies()
+    h2d_ms = time_loop(torch, lambda: copies(True, False), 10)
+    d2h_ms = time_loop(torch, lambda: copies(False, True), 10)
+    both_ms = time_loop(torch, lambda: copies(True, True), 10)
+
     # ---- max over ranks
     ms_total, e2e_ms = reduce_max([ms_total, e2e_ms], device)
     ms_step = ms_total / args.steps
@@ -507,7 +650,8 @@ def run_gpu(args):
     attn_tflops = kf / (attn_ms * 1e-3) / 1e12
     rbytes = routing_bytes(s) / share
     route_gbs = rbytes / (route_ms * 1e-3) / 1e9
-    peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak_b = peaks["bf16_tflops"]
+    peak_s = peaks.get("bf16_tflops_sustained", peak_b)
     out = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -558,11 +702,12 @@ def run_gpu(args):
             "kernel": ("attn_pp_kernel (sparse walk, kept blocks)" if (s.T, s.d) == (128, 128)
                        else f"attn_fwd_kernel<d={s.d},T={s.T}> (sparse walk, kept blocks)"),
             "achieved": round(attn_tflops, 2),
-            "peak": peak_t,
-            "peak_kind": f"bf16 sustained ({peak_kind})",
+            "peak": peak_b,
+            "peak_kind": f"bf16 burst ({peak_kind}): the kernel is timed per launch",
             "unit": "TFLOP/s",
-            "frac": round(attn_tflops / peak_t, 4),
-            "frac_of_burst": round(attn_tflops / peaks["bf16_tflops"], 4),
+            "frac": round(attn_tflops / peak_b, 4),
+            "frac_of_sustained": round(attn_tflops / peak_s, 4),
+            "sustained_peak": peak_s,
             "traffic": attn_traffic() if s.P == 48 and cfg == 3 and share == 1 else None,
         },
         "routing_roofline": {
@@ -576,22 +721,60 @@ def run_gpu(args):
             "ms_per_step": round(e2e_ms, 4),
             "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h),
+            "copies_alone_ms": {"h2d": round(h2d_ms, 4), "d2h": round(d2h_ms, 4),
+                                "both": round(both_ms, 4)},
+            "h2d_gbs": round(h2d / (h2d_ms * 1e-3) / 1e9, 1),
+            "d2h_gbs": round(d2h / (d2h_ms * 1e-3) / 1e9, 1),
             "note": "past KV cache resident; per step the chunk's Q/K/V, depth and camera go "
                     "host->device and O comes back, on copy streams overlapped with the previous "
-                    "/ next step's compute (double-buffered)",
+                    "/ next step's compute (double-buffered); copies_alone_ms times the same "
+                    "copies with no compute",
             "o_matches_device": h_o_ok,
         },
         "gpu_launches": w.launches_per_step * args.steps,
         "device_status": status,
         "clocks": clocks,
     }
+
+    extras = world == 1 and not args.no_extras and cfg == 3 and args.P in (None, 48)
+    checks = []
+    if extras:
+        # ---- rollout-length sweep (workload 4) and the 30-layer pipeline (workload 5)
+        sweep = []
+        for P in SWEEP_P:
+            rec, chk = sweep_point(torch, vx, device, P, max(3, min(10, args.steps // 20)), peaks,
+                                   w.status)
+            sweep.append(rec)
+            checks.append(chk)
+            torch.cuda.empty_cache()
+        out["sweep"] = sweep
+        pipe = pipeline_measure(torch, vx, device, layers=30, steps=3, warmup=3, seed=1005)
+        out["pipeline"] = {key: pipe[key] for key in (
+            "layers", "ms_per_step", "tflops_kept", "geometry_ms", "geometry_done_after_ms",
+            "layer0_routing_done_after_ms", "geometry_exposed_ms", "interleaved_async_step_ms",
+            "interleaved_serial_step_ms")}
+        out["pipeline"]["workload"] = pipe["workload"]
+        out["gpu_launches_outside_timed_region"] = "sweep and pipeline records are timed separately"
+        out["device_status"] = int(w.status.item())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        est, took, desc = oracle_sample(case)
-        out["cpu_baseline"] = {
-            "value": round(kf / est / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_threads(),
-            "kind": "oracle", "sample": desc, "sample_seconds": round(took, 2),
-            "est_step_seconds": round(est, 2),
-        }
+        # the reference arm's sample, repeated for about 10 s of host work (all
+        # threads), then for about 2 s on one thread
+        r = oracle_repeated(case, 10.0)
+        r1 = oracle_single_thread(case)
+        out["cpu_baseline"] = baseline_record(kf, r, r1)
+        # the sampled head's selection against the GPU's, and head 0 of every sweep point
+        ties = {"chunk 48 (workload 3), head 0": selection_ties(gpu_idx[:, :1], r["idx"],
+                                                                 r["s_mod"], s.m)}
+        if extras:
+            from oracle import velox_oracle as vo
+            for chk in checks:
+                cs = chk["shape"]
+                qh = chk["q"].view(torch.int16).numpy().view(np.uint16)
+                kh = chk["k"].view(torch.int16).numpy().view(np.uint16)
+                want, s_mod = vo.route_topk(qh, kh, chk["counts"], cs.alpha, cs.topk, cs.T)
+                ties[f"P = {cs.P} (workload 4), head 0"] = selection_ties(chk["idx"], want, s_mod,
+                                                                           cs.m)
+        out["selection_vs_oracle"] = ties
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -622,24 +805,16 @@ def layer_inputs_on_device(torch, case, layers: int, device, seed: int):
     return w0, qs, ks, vs
 
 
-def run_pipeline(args):
+def pipeline_measure(torch, vx, device, layers: int, steps: int, warmup: int, seed: int) -> dict:
     """One denoising step of the 30-layer pipeline at chunk 48: the geometry
     (recency-priority multiwarp of the 48 past depth maps -> slices -> overlap
     counts) runs on a side stream while layer 0 pools its keys; layer 0's
-    selection waits for the counts; then routing + attention for every layer."""
-    import torch
-    from geometry_routed_block_b200 import velox as vx
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    layers = args.layers
-    case = synth.make_case(5, seed=1005 + rank, layers=1)
+    selection waits for the counts; then routing + attention for every layer.
+    Returns the timings, the geometry's exposure and the clocks."""
+    case = synth.make_case(5, seed=seed, layers=1)
     s = case.shape
     s.layers = layers
-    w, qs, ks, vs = layer_inputs_on_device(torch, case, layers, device, 1005 + rank)
-    peaks, peak_kind = load_peaks()
+    w, qs, ks, vs = layer_inputs_on_device(torch, case, layers, device, seed)
 
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
     past_depth = dev(case.past_depth[0])
@@ -691,13 +866,13 @@ def run_pipeline(args):
         for l in range(layers):
             layer(l)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         step_async()
     step_serial()
     torch.cuda.synchronize()
-    steps = max(1, args.steps)
+    steps = max(1, steps)
     # the timed region: K whole steps with the geometry in flight on the side stream
-    with ClockSampler(local) as clk:
+    with ClockSampler(device.index or 0) as clk:
         t_async = time_loop(torch, step_async, steps)
     clocks = clk.summary()
     # exposure, per step, from events: when the geometry is done vs when layer 0's
@@ -728,15 +903,11 @@ def run_pipeline(args):
     t_geo = g0.elapsed_time(g1) / 20
     med = statistics.median
     kf = kept_flops(s) * layers
-    value = world * kf / (t_async * 1e-3) / 1e12
     out = {
-        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
-        "steps": steps, "warmup": args.warmup, "ms_per_step": round(t_async, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": f"denoising step, {layers} layers x " + workload_desc(s)
-                   + "; current depth from the multiwarp of the past depth maps",
-                   "l2": "inputs larger than L2; no flush"},
+        "layers": layers, "steps": steps, "ms_per_step": round(t_async, 4),
+        "tflops_kept": round(kf / (t_async * 1e-3) / 1e12, 3), "kept_flops": kf,
+        "workload": f"denoising step, {layers} layers x " + workload_desc(s)
+                    + "; current depth from the multiwarp of the past depth maps",
         "geometry_ms": round(t_geo, 4),
         "geometry_done_after_ms": round(med(geo_done), 4),
         "layer0_routing_done_after_ms": round(med(route0_done), 4),
@@ -746,6 +917,32 @@ def run_pipeline(args):
         "gpu_launches": (7 + 4 * layers) * steps,
         "device_status": int(w.status.item()),
         "clocks": clocks,
+    }
+    del qs, ks, vs, w
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_pipeline(args):
+    """The 30-layer pipeline (workload 5) as its own bench line."""
+    import torch
+    from geometry_routed_block_b200 import velox as vx
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    r = pipeline_measure(torch, vx, device, args.layers, args.steps, args.warmup, 1005 + rank)
+    out = {
+        "metric": METRIC, "value": round(world * r["tflops_kept"], 3), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": r["steps"], "warmup": args.warmup,
+        "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": r["workload"], "l2": "inputs larger than L2; no flush"},
+        **{k: r[k] for k in ("geometry_ms", "geometry_done_after_ms",
+                             "layer0_routing_done_after_ms", "geometry_exposed_ms",
+                             "interleaved_async_step_ms", "interleaved_serial_step_ms",
+                             "gpu_launches", "device_status", "clocks")},
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
@@ -1070,6 +1267,10 @@ def run_overlap(args):
 
 
 def run_reference(args):
+    """The reference arm: the fp64 CPU oracle (the method's pages publish no
+    code) on the host cores. Each step is one bounded sample of the workload
+    (oracle_sample); the line reports the time a sample really took and the
+    whole step extrapolated from it, flagged as such."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
@@ -1079,26 +1280,30 @@ def run_reference(args):
     s = synth.shape_for(cfg, P=args.P)
     case.shape = s
     kf = kept_flops(s)
-    # rows per step sized so that warm-up + K steps stay within a few minutes
-    n_rows = max(1, min(s.m, (3 * s.m) // max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(case, n_rows=n_rows)
-    ests, took = [], 0.0
-    for _ in range(args.steps):
-        est, t, desc = oracle_sample(case, n_rows=n_rows)
-        ests.append(est)
-        took += t
-    est = statistics.mean(ests)
-    value = kf / est / 1e12
+        oracle_sample(case)
+    samples = [oracle_sample(case) for _ in range(args.steps)]
+    r = {key: statistics.mean(x[key] for x in samples)
+         for key in ("geometry_s", "routing_s_per_head", "attention_s_per_query_block",
+                     "sample_s", "est_step_s")}
+    r["desc"] = samples[0]["desc"]
+    r["repeats"] = len(samples)
+    r1 = oracle_single_thread(case)
+    value = kf / r["est_step_s"] / 1e12
     out = {
         "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est * 1e3, 1),
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(r["sample_s"] * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
+        "extrapolated": True,
+        "est_full_step_ms": round(r["est_step_s"] * 1e3, 1),
         "config": {"workload": workload_desc(s), "l2": "n/a (host)",
-                   "parallelism": "host cores, rank 0 only"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_threads(),
-                         "kind": "oracle", "sample": desc},
+                   "parallelism": "host cores, rank 0 only",
+                   "step": "one bounded sample of the workload per step (ms_per_step is its "
+                           "measured time); value is the whole step extrapolated from the "
+                           "sample (est_full_step_ms)"},
+        "cpu_baseline": baseline_record(kf, r, r1),
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -1120,9 +1325,12 @@ def main():
     ap.add_argument("--T", type=int, default=None, help="block size (sweep workload: 64 or 128)")
     ap.add_argument("--d", type=int, default=None, help="head dim (sweep workload: 64 or 128)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--shard", default="chunks", choices=["chunks", "heads"],
-                    help="multi-GPU: one chunk per GPU (weak scaling) or the heads of one "
-                         "chunk split over the GPUs with an all-gather of O (strong scaling)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="leave the sweep and pipeline records out of the default line")
+    ap.add_argument("--shard", default="heads", choices=["heads", "chunks"],
+                    help="multi-GPU: the heads of one chunk split over the GPUs with an "
+                         "all-gather of O every step (default, strong scaling), or one "
+                         "independent chunk per GPU with no collective (weak scaling)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

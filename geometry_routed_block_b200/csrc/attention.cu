@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int st = j % nst;
                 const int kb_next = (j + 1 < n) ? fetch(j + 1) : 0;
                 if (j >= nst &&
-                    !mbar_wait(empty(st), ((j / nst) - 1) & 1, abort_flag, WAIT_LIMIT_NS))
+                    !mbar_wait(empty(st), ((j / nst) - 1) & 1, abort_flag, a.wait_ns))
                     break;
                 mbar_arrive_expect_tx(full(st), L::KV_TILE);
 #pragma unroll
@@ -176,15 +176,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (with the skip_mma test hook it issues nothing: every wait on an MMA
+        // completion then runs out, and the kernel reports the timeout)
+        if (lane == 0 && !a.skip_mma) {
             constexpr uint32_t ID_S = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t ID_PV = idesc_bf16_f32(BM, D, false, true);
-            bool ok = mbar_wait(bars.q_full(), 0, abort_flag, WAIT_LIMIT_NS);
+            bool ok = mbar_wait(bars.q_full(), 0, abort_flag, a.wait_ns);
             tc_fence_after();
             auto issue_s = [&](int j) -> bool {
                 const int s = j % KST;
                 const int bi = j & 1;
-                if (!mbar_wait(bars.k_full(s), (j / KST) & 1, abort_flag, WAIT_LIMIT_NS))
+                if (!mbar_wait(bars.k_full(s), (j / KST) & 1, abort_flag, a.wait_ns))
                     return false;
                 // S buffer bi last held P_{j-2}, read by PV_{j-2}, which this
                 // thread issued earlier: MMAs from one thread run in issue order
@@ -208,8 +210,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (j + 1 < n && !issue_s(j + 1)) break;
                 const int s = j % VST;
                 const int bi = j & 1;
-                if (!mbar_wait(bars.v_full(s), (j / VST) & 1, abort_flag, WAIT_LIMIT_NS)) break;
-                if (!mbar_wait(bars.p_full(bi), (j >> 1) & 1, abort_flag, WAIT_LIMIT_NS)) break;
+                if (!mbar_wait(bars.v_full(s), (j / VST) & 1, abort_flag, a.wait_ns)) break;
+                if (!mbar_wait(bars.p_full(bi), (j >> 1) & 1, abort_flag, a.wait_ns)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
@@ -262,7 +264,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int j = 0; j < n; ++j) {
             const int bi = j & 1;
-            if (!warp_wait(bars.s_full(bi), (j >> 1) & 1, abort_flag)) {
+            if (!warp_wait(bars.s_full(bi), (j >> 1) & 1, abort_flag, a.wait_ns)) {
                 ok = false;
                 break;
             }
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (__any_sync(0xffffffffu, resc)) {
                 // O must hold PV_{j-1} before it is rescaled in place
-                if (!warp_wait(bars.pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) {
+                if (!warp_wait(bars.pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.p_full(bi));  // P_j and (rescaled) O are ready
         }
-        if (ok && n > 0 && warp_wait(bars.pv_done((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag)) {
+        if (ok && n > 0 && warp_wait(bars.pv_done((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, a.wait_ns)) {
             tc_fence_after();
             const float inv = 1.f / l_run;
             const bool store = row < a.T;

@@ -44,11 +44,6 @@ constexpr int PP_VST = 2;
 constexpr int PP_WARP_TMA_K = 8;
 constexpr int PP_WARP_MMA = 9;
 constexpr int PP_WARP_TMA_V = 10;
-// Every exponential goes to the ex2 unit here: with two blocks in flight the
-// softmax has slack, and moving part of the exponentials to the FMA pipe
-// (as the single-block kernel does) only adds issue pressure (measured on the
-// chunk-48 walk: 0/8 of the pairs emulated 1,171 TFLOP/s, 3/8 1,152, 4/8 1,091).
-constexpr unsigned PP_EMU_MASK = 0x00;
 
 struct PPLayout {
     static constexpr int TILE = 128 * 128 * 2;  // a Q, K or V tile: 128 rows x 128 bf16
@@ -80,19 +75,19 @@ struct PPBars {
     __device__ uint32_t pv_done(int t) const { return base + 8 * (R + 4 + t); }
 };
 
-// exponentials of 64 scores (one half row) in place, sums into sum2
+// exponentials of 64 scores (one half row) in place, sums into sum2. Every
+// exponential goes to the ex2 unit here: with two blocks in flight the
+// softmax has slack, and moving part of them to the FMA pipe (as the
+// single-block kernel does) only adds issue pressure (measured on the chunk-48
+// walk: none of the pairs emulated 1,171 TFLOP/s, 3/8 1,152, 4/8 1,091).
 __device__ __forceinline__ void exp_half(float* s, float sl2, float m, float2* sum2) {
     const float2 sc2 = make_float2(sl2, sl2);
     const float2 ng2 = make_float2(-m, -m);
 #pragma unroll
     for (int i = 0; i < 64; i += 2) {
         float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), sc2, ng2);
-        if ((PP_EMU_MASK >> ((i >> 1) & 7)) & 1) {
-            x = exp2_poly2(x);
-        } else {
-            x.x = ex2_approx(x.x);
-            x.y = ex2_approx(x.y);
-        }
+        x.x = ex2_approx(x.x);
+        x.y = ex2_approx(x.y);
         s[i] = x.x;
         s[i + 1] = x.y;
         sum2[(i >> 1) & 3] = __fadd2_rn(sum2[(i >> 1) & 3], x);
@@ -213,7 +208,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                         bar = empty(st);
                         par = static_cast<uint32_t>(((l / nst) - 1) & 1);
                     }
-                    if (!mbar_wait(bar, par, abort_flag, WAIT_LIMIT_NS)) break;
+                    if (!mbar_wait(bar, par, abort_flag, a.wait_ns)) break;
                 }
                 mbar_arrive_expect_tx(full(st), L::TILE);
 #pragma unroll
@@ -230,15 +225,17 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
         }
     } else if (warp == PP_WARP_MMA) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (with the skip_mma test hook it issues nothing: every wait on an MMA
+        // completion then runs out, and the kernel reports the timeout)
+        if (lane == 0 && !a.skip_mma) {
             constexpr uint32_t ID_S = idesc_bf16_f32(128, PP_BN, false, false);
             constexpr uint32_t ID_PV = idesc_bf16_f32(128, PP_D, false, true);
-            bool ok = mbar_wait(bars.q_full(), 0, abort_flag, WAIT_LIMIT_NS);
+            bool ok = mbar_wait(bars.q_full(), 0, abort_flag, a.wait_ns);
             tc_fence_after();
             int kl = 0, vl = 0;
             auto issue_s = [&](int t) -> bool {
                 const int st = kl % PP_KST;
-                if (!mbar_wait(bars.k_full(st), (kl / PP_KST) & 1, abort_flag, WAIT_LIMIT_NS))
+                if (!mbar_wait(bars.k_full(st), (kl / PP_KST) & 1, abort_flag, a.wait_ns))
                     return false;
                 tc_fence_after();
                 const uint32_t d = tmem + t * 128;
@@ -256,9 +253,9 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             };
             auto issue_pv = [&](int t, int i) -> bool {
                 const int st = vl % PP_VST;
-                if (!mbar_wait(bars.v_full(st), (vl / PP_VST) & 1, abort_flag, WAIT_LIMIT_NS))
+                if (!mbar_wait(bars.v_full(st), (vl / PP_VST) & 1, abort_flag, a.wait_ns))
                     return false;
-                if (!mbar_wait(bars.p_full(t), i & 1, abort_flag, WAIT_LIMIT_NS)) return false;
+                if (!mbar_wait(bars.p_full(t), i & 1, abort_flag, a.wait_ns)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < PP_BN / 16; ++kk) {
@@ -294,7 +291,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
         float l_run = 0.f;
         bool ok = true;
         for (int i = 0; i < n; ++i) {
-            if (!warp_wait(bars.s_full(t), i & 1, abort_flag)) {
+            if (!warp_wait(bars.s_full(t), i & 1, abort_flag, a.wait_ns)) {
                 ok = false;
                 break;
             }
@@ -347,7 +344,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             const float rs = s03.x + s03.y;
             if (__any_sync(0xffffffffu, resc)) {
                 // O must hold P(i-1) V(i-1) before it is rescaled in place
-                if (!warp_wait(bars.pv_done(t), (i - 1) & 1, abort_flag)) {
+                if (!warp_wait(bars.pv_done(t), (i - 1) & 1, abort_flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -372,7 +369,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.p_full(t));  // P(i) and (rescaled) O ready
         }
-        if (ok && n > 0 && warp_wait(bars.pv_done(t), (n - 1) & 1, abort_flag)) {
+        if (ok && n > 0 && warp_wait(bars.pv_done(t), (n - 1) & 1, abort_flag, a.wait_ns)) {
             tc_fence_after();
             const float inv = 1.f / l_run;
             const size_t grow = static_cast<size_t>(bh) * a.Nq + static_cast<size_t>(qb) * PP_BN + row;

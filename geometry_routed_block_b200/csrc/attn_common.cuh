@@ -16,7 +16,6 @@
 
 namespace velox {
 
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr float RESCALE_THRESHOLD = 8.0f;          // log2 units
 
 namespace {
@@ -73,8 +72,9 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 }
 
 // bounded wait, made uniform across the warp (a warp leaves together)
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-    bool ok = mbar_wait(bar, parity, abort, WAIT_LIMIT_NS);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns) {
+    bool ok = mbar_wait(bar, parity, abort, limit_ns);
     return __all_sync(0xffffffffu, ok);
 }
 

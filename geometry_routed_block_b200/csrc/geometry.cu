@@ -288,26 +288,30 @@ int overlap_launch(const float* depth, const velox_slice_t* cur, const velox_sli
     return launch_status();
 }
 
-size_t multiwarp_ws_bytes(int HW) {
-    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    return 2 * up(static_cast<size_t>(HW) * 8) + up(static_cast<size_t>(HW) * 4);
-}
+// Scratch of the multiwarp for an HW-pixel grid: z_min and the winner's depth
+// (64-bit each) and the winning chunk (32-bit), each array 256-byte aligned.
+constexpr size_t mw_up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+constexpr size_t mw_ws_bytes(size_t HW) { return 2 * mw_up256(HW * 8) + mw_up256(HW * 4); }
+
+size_t multiwarp_ws_bytes(int HW) { return mw_ws_bytes(static_cast<size_t>(HW)); }
 
 int multiwarp_launch(const float* past_depth, const velox_slice_t* past, const velox_slice_t* cur,
                      int P, int Hp, int Wp, float rel_tol, float* out, void* ws, cudaStream_t st) {
     const int HW = Hp * Wp;
-    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     char* w = static_cast<char*>(ws);
     auto* zmin = reinterpret_cast<unsigned long long*>(w);
-    auto* zbest = reinterpret_cast<unsigned long long*>(w + up(static_cast<size_t>(HW) * 8));
-    auto* jwin = reinterpret_cast<int*>(w + 2 * up(static_cast<size_t>(HW) * 8));
+    auto* zbest = reinterpret_cast<unsigned long long*>(w + mw_up256(static_cast<size_t>(HW) * 8));
+    auto* jwin = reinterpret_cast<int*>(w + 2 * mw_up256(static_cast<size_t>(HW) * 8));
+    // n = P * HW < 2^31 (checked by the callers); block counts in 64-bit arithmetic
     const int n = P * HW;
+    const unsigned pix_blocks = static_cast<unsigned>((static_cast<long long>(HW) + 255) / 256);
+    const unsigned pt_blocks = static_cast<unsigned>((static_cast<long long>(n) + 255) / 256);
     const double factor = 1.0 + static_cast<double>(rel_tol);
-    mw_init_kernel<<<(HW + 255) / 256, 256, 0, st>>>(zmin, jwin, zbest, HW);
-    mw_zmin_kernel<<<(n + 255) / 256, 256, 0, st>>>(past_depth, past, cur, n, Hp, Wp, zmin);
-    mw_winner_kernel<<<(n + 255) / 256, 256, 0, st>>>(past_depth, past, cur, n, Hp, Wp, factor, zmin, jwin);
-    mw_depth_kernel<<<(n + 255) / 256, 256, 0, st>>>(past_depth, past, cur, n, Hp, Wp, jwin, zbest);
-    mw_final_kernel<<<(HW + 255) / 256, 256, 0, st>>>(zbest, HW, out);
+    mw_init_kernel<<<pix_blocks, 256, 0, st>>>(zmin, jwin, zbest, HW);
+    mw_zmin_kernel<<<pt_blocks, 256, 0, st>>>(past_depth, past, cur, n, Hp, Wp, zmin);
+    mw_winner_kernel<<<pt_blocks, 256, 0, st>>>(past_depth, past, cur, n, Hp, Wp, factor, zmin, jwin);
+    mw_depth_kernel<<<pt_blocks, 256, 0, st>>>(past_depth, past, cur, n, Hp, Wp, jwin, zbest);
+    mw_final_kernel<<<pix_blocks, 256, 0, st>>>(zbest, HW, out);
     return launch_status();
 }
 
@@ -354,33 +358,76 @@ int cast_bf16_launch(const float* x, uint16_t* y, size_t n, cudaStream_t st) {
 // memory. Each GPU that loads the library holds the array until the process
 // exits. All calls share it, so calls that overlap on the GPU race.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 namespace velox {
 namespace {
 
 constexpr int NOALLOC_MAX_PIXELS = VELOX_MULTIWARP_NOALLOC_MAX_PIXELS;
-constexpr size_t NOALLOC_BYTES =
-    2 * static_cast<size_t>(NOALLOC_MAX_PIXELS) * 8 + static_cast<size_t>(NOALLOC_MAX_PIXELS) * 4;
-constexpr int NOALLOC_MAX_DEVICES = 64;
+// the same layout (and 256-byte rounding) the launch uses to carve the scratch
+constexpr size_t NOALLOC_BYTES = mw_ws_bytes(static_cast<size_t>(NOALLOC_MAX_PIXELS));
+static_assert(NOALLOC_BYTES >= mw_ws_bytes(NOALLOC_MAX_PIXELS), "scratch array too small");
+constexpr int NOALLOC_CACHE = 64;
 
 static __device__ __align__(256) unsigned char g_multiwarp_scratch[NOALLOC_BYTES];
 
-// Device address of the array on the current device. The host-side symbol is
-// only a stand-in; the real address is looked up once per device, with that
-// device current, and cached.
-void* multiwarp_scratch_on_current_device() {
-    static std::mutex mu;
-    static void* addr[NOALLOC_MAX_DEVICES] = {};
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
+// The driver calls that identify the current context (a CUDA context has a
+// process-unique id, so a context created after cudaDeviceReset never matches
+// an older entry even if its handle is reused).
+struct CtxApi {
+    PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+
+const CtxApi& ctx_api() {
+    static CtxApi api;
+    static std::once_flag once;
+    std::call_once(once, [] {
         void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            api.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            api.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    return api;
+}
+
+// Device address of the array in the current context. The host-side symbol is
+// only a stand-in; the real address is looked up with cudaGetSymbolAddress the
+// first time a context calls, and cached under that context's id.
+void* multiwarp_scratch_in_current_context() {
+    static std::mutex mu;
+    static unsigned long long ids[NOALLOC_CACHE] = {};
+    static void* addrs[NOALLOC_CACHE] = {};
+    static int next = 0;
+    const CtxApi& api = ctx_api();
+    if (!api.get_current || !api.get_id) return nullptr;
+    void* p = nullptr;
+    CUcontext ctx = nullptr;
+    if (api.get_current(&ctx) != CUDA_SUCCESS) return nullptr;
+    if (ctx == nullptr) {
+        // no context bound to this thread yet: the runtime lookup binds the
+        // device's primary context
         if (cudaGetSymbolAddress(&p, g_multiwarp_scratch) != cudaSuccess) return nullptr;
-        addr[dev] = p;
+        if (api.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
     }
-    return addr[dev];
+    unsigned long long id = 0;
+    if (api.get_id(ctx, &id) != CUDA_SUCCESS) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < NOALLOC_CACHE; ++i)
+        if (addrs[i] != nullptr && ids[i] == id) return addrs[i];
+    if (p == nullptr && cudaGetSymbolAddress(&p, g_multiwarp_scratch) != cudaSuccess) return nullptr;
+    ids[next] = id;
+    addrs[next] = p;
+    next = (next + 1) % NOALLOC_CACHE;
+    return p;
 }
 
 }  // namespace
@@ -394,7 +441,7 @@ extern "C" int velox_depth_multiwarp_noalloc(const float* past_depth,
     if (P < 1 || Hp < 1 || Wp < 1 || !(rel_tol >= 0.0f) || !isfinite(rel_tol)) return VELOX_EINVAL;
     if (static_cast<long long>(Hp) * Wp > velox::NOALLOC_MAX_PIXELS) return VELOX_EINVAL;
     if (static_cast<long long>(P) * Hp * Wp >= (1ll << 31)) return VELOX_EINVAL;
-    void* scratch = velox::multiwarp_scratch_on_current_device();
+    void* scratch = velox::multiwarp_scratch_in_current_context();
     if (scratch == nullptr) return VELOX_ECUDA;
     // the launch sequence starts by resetting the per-pixel state it uses
     return velox::multiwarp_launch(past_depth, past_cams, cur_cam, P, Hp, Wp, rel_tol, cur_depth,

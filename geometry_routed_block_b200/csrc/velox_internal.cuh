@@ -11,6 +11,10 @@
 
 namespace velox {
 
+// default limit of the attention kernels' bounded waits: 2 s, far above any
+// legitimate wait
+constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;
+
 struct AttnArgs {
     const int32_t* idx;  // [B*H][m][n_sel] or nullptr (dense)
     int n_sel;           // key blocks per query block
@@ -21,6 +25,8 @@ struct AttnArgs {
     int32_t* status;
     const __nv_bfloat16* q;  // set by the launcher
     long long q_rows;        // B * H * Nq
+    unsigned long long wait_ns;  // limit of every bounded wait
+    int skip_mma;                // test hook: the tensor-core issuer issues nothing
 };
 
 int attn_fwd_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B, int d,

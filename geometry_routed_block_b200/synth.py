@@ -358,12 +358,14 @@ def _walk(seed: int, s: Shape) -> Case:
                 slices_given=False)
 
 
-def _loop(cfg: int, seed: int, s: Shape, heads: tuple | None = None) -> Case:
+def _loop(cfg: int, seed: int, s: Shape, heads: tuple | None = None,
+          layer_ids: tuple | None = None) -> Case:
     """Room scene, looping trajectory (period 16), K of past chunk c shifted
     toward the head's query mean by the view-overlap proxy of chunk c.
 
-    `heads` restricts which heads are materialised (the rest are drawn and
-    discarded, so a head's values do not depend on the selection)."""
+    `heads` and `layer_ids` restrict which heads and layers are materialised;
+    every (layer, head) has its own generator, so its values do not depend on
+    the selection."""
     rng = np.random.default_rng(seed)
     scene = room_scene(rng)
     intr = intrinsics(s.Hp, s.Wp, s.fov_deg)
@@ -371,30 +373,30 @@ def _loop(cfg: int, seed: int, s: Shape, heads: tuple | None = None) -> Case:
     depths = np.stack([render_depth(scene, p, intr, s.Hp, s.Wp) for p in poses])
     ov = np.array([view_overlap_proxy(yaws[c], yaws[s.P], s.fov_deg) for c in range(s.P)],
                   dtype=np.float32)
-    L = s.layers
+    lsel = list(range(s.layers)) if layer_ids is None else list(layer_ids)
     hsel = list(range(s.H)) if heads is None else list(heads)
-    q = np.empty((L, s.B, len(hsel), s.Nq, s.d), np.uint16)
-    k = np.empty((L, s.B, len(hsel), s.Nk, s.d), np.uint16)
-    v = np.empty((L, s.B, len(hsel), s.Nk, s.d), np.uint16)
-    mus = [0.5 * _normal(np.random.default_rng([seed, l]), (s.H, s.d)) for l in range(L)]
+    q = np.empty((len(lsel), s.B, len(hsel), s.Nq, s.d), np.uint16)
+    k = np.empty((len(lsel), s.B, len(hsel), s.Nk, s.d), np.uint16)
+    v = np.empty((len(lsel), s.B, len(hsel), s.Nk, s.d), np.uint16)
+    mus = {l: 0.5 * _normal(np.random.default_rng([seed, l]), (s.H, s.d)) for l in lsel}
 
-    def head(l, i, h):
+    def head(li, l, i, h):
         hrng = np.random.default_rng([seed, l, h])
         mu = mus[l][h]
-        q[l, 0, i] = f32_to_bf16_bits(_normal(hrng, (s.Nq, s.d)) + mu)
+        q[li, 0, i] = f32_to_bf16_bits(_normal(hrng, (s.Nq, s.d)) + mu)
         kh = _normal(hrng, (s.P + 1, s.Nq, s.d))
         kh[: s.P] += ov[:, None, None] * mu[None, None, :]
-        k[l, 0, i] = f32_to_bf16_bits(kh.reshape(s.Nk, s.d))
-        v[l, 0, i] = f32_to_bf16_bits(_normal(hrng, (s.Nk, s.d)))
+        k[li, 0, i] = f32_to_bf16_bits(kh.reshape(s.Nk, s.d))
+        v[li, 0, i] = f32_to_bf16_bits(_normal(hrng, (s.Nk, s.d)))
 
-    _parallel_heads(head, [(l, i, h) for l in range(L) for i, h in enumerate(hsel)])
+    _parallel_heads(head, [(li, l, i, h) for li, l in enumerate(lsel) for i, h in enumerate(hsel)])
     past_poses = np.stack(poses[: s.P])
     cams = np.stack([camera_record(p, intr) for p in poses[: s.P]])
     return Case(cfg=cfg, shape=s, seed=seed, q=q, k=k, v=v, cur_depth=depths[s.P][None],
                 cur_cam=camera_record(poses[s.P], intr)[None], past_depth=depths[: s.P][None],
                 past_poses=past_poses[None], past_intr=np.tile(intr, (s.P, 1))[None],
                 past_cams=cams[None], slices_given=False,
-                meta={"view_overlap": ov, "heads": hsel})
+                meta={"view_overlap": ov, "heads": hsel, "layers": lsel})
 
 
 def stress_geometry(B: int, P: int, Hp: int, Wp: int, seed: int, fov_deg: float = 60.0,
@@ -443,16 +445,18 @@ def perturb_depth(depth: np.ndarray, rng: np.random.Generator, noise_sd: float =
 
 def make_case(cfg: int, seed: int | None = None, P: int | None = None, H: int | None = None,
               layers: int | None = None, heads: tuple | None = None, T: int | None = None,
-              d: int | None = None) -> Case:
+              d: int | None = None, layer_ids: tuple | None = None) -> Case:
     """Build workload `cfg` (1..5). Default seed is 1000 + cfg. Workload 4 also
-    takes another block size T or head dim d."""
+    takes another block size T or head dim d. For workloads 3-5, `heads` and
+    `layer_ids` materialise only those heads and layers (q/k/v are then
+    [len(layer_ids), B, len(heads), N, d])."""
     seed = 1000 + cfg if seed is None else seed
     if cfg == 1:
         return _tiny(seed)
     s = shape_for(cfg, P=P, H=H, layers=layers, T=T, d=d)
     if cfg == 2:
         return _walk(seed, s)
-    return _loop(cfg, seed, s, heads=heads)
+    return _loop(cfg, seed, s, heads=heads, layer_ids=layer_ids)
 
 
 def geometry_only(cfg: int, seed: int | None = None, P: int | None = None):

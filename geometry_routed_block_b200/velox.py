@@ -27,6 +27,7 @@ VELOX_ETIMEOUT = -4
 VELOX_EBOUNDS = -5
 VELOX_STATUS_BAD_INDEX = 1
 VELOX_STATUS_TIMEOUT = 2
+VELOX_TEST_SKIP_MMA = 1
 VELOX_BF16 = 0
 VELOX_F32 = 1
 CAM_FLOATS = 18
@@ -45,6 +46,9 @@ SIGNATURES = {
                                   _vp, _c_float, _c_int, _vp, _vp, _c_size, _vp, _vp]),
     "velox_sparse_attn_fwd": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                        _c_int, _c_int, _c_float, _vp, _vp, _vp, _vp]),
+    "velox_sparse_attn_fwd_test": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
+                                            _c_int, _c_int, _c_int, _c_float, _vp, _vp, _vp,
+                                            ctypes.c_double, _c_int, _vp]),
     "velox_depth_multiwarp_workspace_size": (_c_size, [_c_int, _c_int]),
     "velox_depth_multiwarp": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_float, _vp, _vp,
                                        _c_size, _vp]),
@@ -275,6 +279,30 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torc
                                      T, float(scale), _ptr(out), _ptr(lse), _ptr(status),
                                      _stream(stream)), "velox_sparse_attn_fwd")
     return out, lse
+
+
+def sparse_attn_fwd_test(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         idx: torch.Tensor | None, T: int, status: torch.Tensor,
+                         wait_limit_s: float, flags: int, out: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """sparse_attn_fwd through the test entry point (bounded-wait limit and
+    failure-injection flags); returns O (unwritten when the waits ran out)."""
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _expect(t, torch.bfloat16, n)
+    _expect(status, torch.int32, "status")
+    topk = 0
+    if idx is not None:
+        _expect(idx, torch.int32, "idx")
+        topk = idx.shape[-1]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.velox_sparse_attn_fwd_test(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), topk, B, H, Nq, Nk,
+                                          d, T, float(1.0 / math.sqrt(d)), _ptr(out), None,
+                                          _ptr(status), float(wait_limit_s), int(flags),
+                                          _stream(stream)), "velox_sparse_attn_fwd_test")
+    return out
 
 
 def fp64_fma_bench(out: torch.Tensor, blocks: int, threads: int, iters: int, stream=None) -> int:

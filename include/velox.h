@@ -22,7 +22,9 @@
  *   - Every pointer argument is a DEVICE pointer owned by the caller unless
  *     stated otherwise. The library never allocates, frees or synchronises;
  *     scratch memory, where an operation needs it, is passed in by the caller
- *     (sizes from the matching *_workspace_size function).
+ *     (sizes from the matching *_workspace_size function). The one exception
+ *     is velox_depth_multiwarp_noalloc, whose scratch is a fixed array owned
+ *     by the library.
  *   - Tensors are dense, row-major, innermost dimension last. Q/K/V/O use the
  *     layout [B][H][N][d]. In the KV cache the past chunks come first (oldest
  *     first) and the current chunk occupies the last Nq keys.
@@ -30,7 +32,9 @@
  *     default stream): it validates its arguments, enqueues kernels and returns.
  *     A rejected call (VELOX_EINVAL / VELOX_EUNSUPPORTED) launches nothing.
  *   - Calls hold no global state and may run concurrently on distinct streams
- *     with distinct outputs and workspaces.
+ *     with distinct outputs and workspaces -- except velox_depth_multiwarp_noalloc:
+ *     all its calls share the library's scratch array, so they must not
+ *     overlap on the GPU (serialise them, e.g. on one stream).
  *   - `status` arguments (may be NULL) point to one device int32 that kernels
  *     OR VELOX_STATUS_* bits into when they detect a bad index or give up a
  *     bounded wait; the caller zeroes it and reads it back.
@@ -178,6 +182,31 @@ VELOX_API int velox_sparse_attn_fwd(const void* q, const void* k, const void* v,
                           int topk, int B, int H, int Nq, int Nk, int d, int T, float scale,
                           void* o, float* lse, int32_t* status, void* stream);
 
+/* test-hook flags of velox_sparse_attn_fwd_test */
+#define VELOX_TEST_SKIP_MMA 1
+
+/*
+ * velox_sparse_attn_fwd with two test hooks for its failure path; not a step
+ * of the method. Every wait inside the attention kernels is bounded: a wait
+ * that runs out sets VELOX_STATUS_TIMEOUT in *status, the CTA's other waits
+ * give up, copies already in flight are drained and the kernel returns, so
+ * the device stays usable. This entry point lets a test reach that path
+ * without a fault:
+ *   wait_limit_s  limit of each bounded wait, in seconds, in [1e-3, 10]
+ *                 (velox_sparse_attn_fwd uses 2 s);
+ *   flags         VELOX_TEST_SKIP_MMA: the tensor-core issuer issues nothing,
+ *                 so no MMA completion ever arrives and the waits on them run
+ *                 out (no MMA is in flight when tensor memory is freed); the
+ *                 output is left unwritten. 0: a normal call.
+ * Other arguments, results and errors are those of velox_sparse_attn_fwd;
+ * VELOX_EINVAL also for a limit outside the range or an unknown flag.
+ */
+VELOX_API int velox_sparse_attn_fwd_test(const void* q, const void* k, const void* v,
+                                         const int32_t* idx, int topk, int B, int H, int Nq,
+                                         int Nk, int d, int T, float scale, void* o, float* lse,
+                                         int32_t* status, double wait_limit_s, int flags,
+                                         void* stream);
+
 /*
  * Pooled-key cache (an incremental form of the routing's key pooling; the
  * block importance the model computes in each layer, "Tiefenanalyse" step 3,
@@ -250,9 +279,12 @@ VELOX_API int velox_depth_multiwarp(const float* past_depth, const velox_slice_t
  * process exits.
  *   - Hp * Wp above VELOX_MULTIWARP_NOALLOC_MAX_PIXELS returns VELOX_EINVAL and
  *     launches nothing.
- *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture. A failed lookup returns VELOX_ECUDA.
+ *   - The first call in a CUDA context (normally: the first call on a device,
+ *     whose primary context the runtime uses) looks up the array's device
+ *     address with that context current and caches it under the context's
+ *     id; make that first call before any stream capture. A context created
+ *     later for the same device (after cudaDeviceReset, say) gets its own
+ *     lookup. A failed lookup returns VELOX_ECUDA.
  *   - Every call resets the scratch it uses before reading it, but all calls
  *     share one array: calls whose kernels overlap on the GPU (e.g. on two
  *     streams at once) race and give wrong depths. Serialise them.

@@ -26,3 +26,8 @@ def test_reference_arm_prints_one_contract_line():
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"]
     assert "workload" in d["config"]
+    # the sample really ran once per step; the whole step is an extrapolation, flagged
+    assert d["extrapolated"] is True and d["est_full_step_ms"] > d["ms_per_step"] > 0
+    cb = d["cpu_baseline"]
+    assert cb["extrapolated"] is True and cb["single_thread"]["cores"] == 1
+    assert cb["attention_s_per_query_block"] > 0 and cb["routing_s_per_head"] > 0

@@ -1,6 +1,7 @@
 """The multi-GPU host logic of bench.py on CPU: two gloo ranks (127.0.0.1).
-Each rank times its own chunk; the job time is the max over ranks and the
-whole-job rate counts every rank's work (weak scaling, no data collective)."""
+The job time is the max over ranks and the whole-job rate counts every rank's
+work; the default multi-GPU mode splits the heads of one chunk over the ranks
+and all-gathers O in place; the other mode runs one chunk per rank."""
 import os
 import socket
 import sys
@@ -63,11 +64,19 @@ def _heads_main(rank, world, port, out):
     from datetime import timedelta
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
     import bench
-    B, H, N, d = 2, 24, 8, 4
-    full = torch.arange(B * H * N * d, dtype=torch.float32).view(B, H, N, d)
-    h0, h1 = bench.head_range(H, world, rank)
-    got = bench.gather_heads(full[:, h0:h1].clone(), world)
-    out[rank] = ((h0, h1), bool(torch.equal(got, full)))
+    ok = []
+    for B in (1, 2):
+        H, N, d = 24, 8, 4
+        full = torch.arange(B * H * N * d, dtype=torch.float32).view(B, H, N, d)
+        h0, h1 = bench.head_range(H, world, rank)
+        # this rank's heads are written into its slice of the gathered buffer,
+        # which the all-gather then fills in place
+        o_all = torch.full((world * B, h1 - h0, N, d), -1.0)
+        mine = o_all[rank * B:(rank + 1) * B]
+        mine.copy_(full[:, h0:h1])
+        got = bench.gather_heads(o_all, mine, world)
+        ok.append(bool(torch.equal(got, full)))
+    out[rank] = ((h0, h1), all(ok))
     dist.barrier()
     dist.destroy_process_group()
 
