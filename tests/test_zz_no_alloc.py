@@ -78,7 +78,9 @@ def test_noalloc_multiwarp_at_the_pixel_limit():
         assert rc == 0, vx.strerror(rc)
         torch.cuda.synchronize()
         assert np.array_equal(got.cpu().numpy(), want.cpu().numpy(), equal_nan=True)
-    assert torch.isfinite(want).float().mean().item() > 0.5
+    # a forward splat of six maps at this resolution leaves holes; enough pixels
+    # are covered that the comparison is not trivial
+    assert torch.isfinite(want).float().mean().item() > 0.3
 
 
 def test_noalloc_multiwarp_rejects_grids_above_the_limit():
