@@ -29,7 +29,10 @@
 // Ordering: S_t(i+1) overwrites the P_t(i) that O_t += P_t(i) V_t(i) reads;
 // the issuing thread issues the P V first, and MMAs from one thread execute
 // in issue order. A commit tracks every MMA issued before it, so S_t(i+1)
-// complete implies O_t += P_t(i) V_t(i) complete.
+// complete implies O_t += P_t(i) V_t(i) complete. P V is issued in two halves
+// of the keys: the softmax stores the P of keys 64-127 first (their scores are
+// still in registers after the row max) and releases them at once, so the
+// tensor core works on that half while the softmax computes the other.
 #include "attn_common.cuh"
 
 namespace velox {
@@ -51,8 +54,9 @@ struct PPLayout {
     static constexpr int OFF_K = 2 * TILE;
     static constexpr int OFF_V = OFF_K + PP_KST * TILE;
     static constexpr int OFF_BAR = OFF_V + PP_VST * TILE;
-    // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2], pv_done[2]
-    static constexpr int NBAR = 1 + 2 * PP_KST + 2 * PP_VST + 6;
+    // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2],
+    // pv_done[2], p_half[2], mma_drain
+    static constexpr int NBAR = 1 + 2 * PP_KST + 2 * PP_VST + 9;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
@@ -73,6 +77,8 @@ struct PPBars {
     __device__ uint32_t s_full(int t) const { return base + 8 * (R + t); }
     __device__ uint32_t p_full(int t) const { return base + 8 * (R + 2 + t); }
     __device__ uint32_t pv_done(int t) const { return base + 8 * (R + 4 + t); }
+    __device__ uint32_t p_half(int t) const { return base + 8 * (R + 6 + t); }
+    __device__ uint32_t mma_drain() const { return base + 8 * (R + 8); }
 };
 
 // exponentials of 64 scores (one half row) in place, sums into sum2. Every
@@ -137,8 +143,10 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(bars.s_full(t), 1);
             mbar_init(bars.p_full(t), 4);  // one elected arrive per softmax warp
+            mbar_init(bars.p_half(t), 4);
             mbar_init(bars.pv_done(t), 1);
         }
+        mbar_init(bars.mma_drain(), 1);
         fence_mbar_init();
     }
     if (warp == PP_WARP_MMA) {
@@ -251,19 +259,28 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                 ++kl;
                 return true;
             };
+            // O_t += P_t(i) V_t(i) in two halves of the keys: keys 64-127 as soon as
+            // the softmax has stored their P (p_half), keys 0-63 once all of P is
+            // stored (p_full), so the tensor core starts on P V while the softmax
+            // still computes the rest of P
             auto issue_pv = [&](int t, int i) -> bool {
                 const int st = vl % PP_VST;
                 if (!mbar_wait(bars.v_full(st), (vl / PP_VST) & 1, abort_flag, a.wait_ns))
                     return false;
-                if (!mbar_wait(bars.p_full(t), i & 1, abort_flag, a.wait_ns)) return false;
-                tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < PP_BN / 16; ++kk) {
-                    const uint32_t at = tmem + t * 128 + L::P_OFF + kk * 8;
-                    const uint64_t bd = smem_desc_sw128(
-                        sbase + L::OFF_V + st * L::TILE + kk * (16 * 128), PP_BN * 128);
-                    mma_bf16_ts(tmem + L::TMEM_O + t * 128, at, bd, ID_PV,
-                                (i > 0 || kk > 0) ? 1u : 0u);
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t bar = h == 0 ? bars.p_half(t) : bars.p_full(t);
+                    if (!mbar_wait(bar, i & 1, abort_flag, a.wait_ns)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int j = 0; j < PP_BN / 32; ++j) {
+                        const int kk = (h == 0 ? PP_BN / 32 : 0) + j;
+                        const uint32_t at = tmem + t * 128 + L::P_OFF + kk * 8;
+                        const uint64_t bd = smem_desc_sw128(
+                            sbase + L::OFF_V + st * L::TILE + kk * (16 * 128), PP_BN * 128);
+                        mma_bf16_ts(tmem + L::TMEM_O + t * 128, at, bd, ID_PV,
+                                    (i > 0 || h > 0 || j > 0) ? 1u : 0u);
+                    }
                 }
                 if (!has_b) mma_commit(bars.v_empty(st));
                 mma_commit(bars.pv_done(t));
@@ -277,6 +294,10 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                 if (!issue_pv(0, i)) break;
                 if (has_b && i == n - 1) issue_pv(1, i);
             }
+            // every MMA issued above has completed before this thread leaves (on
+            // an abort, too), so none is in flight when tensor memory is freed
+            mma_commit(bars.mma_drain());
+            drain_wait(bars.mma_drain(), 0);
         }
     } else if (warp < 8 && (warp < 4 || has_b)) {
         // ------------------------------------------------------------ softmax warpgroups
@@ -322,34 +343,16 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                 m_new = mx;
                 resc = (i > 0);
             }
-            // pass 2: the second half is in registers; its P goes to columns 96-127
-            // (S columns already read), then the first half is read again and its
-            // P goes to columns 64-95
-            float2 sum2[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) sum2[k] = make_float2(0.f, 0.f);
-            exp_half(s, sl2, m_new, sum2);
-            store_p_half(t_s + L::P_OFF + 32, s);
-            tmem_ld32(t_s, s);
-            tmem_ld32(t_s + 32, s + 32);
-            tmem_wait_ld();
-            reg_fence32(s);
-            reg_fence32(s + 32);
-            exp_half(s, sl2, m_new, sum2);
-            store_p_half(t_s + L::P_OFF, s);
-            tmem_wait_st();
-            const float2 s01 = __fadd2_rn(sum2[0], sum2[1]);
-            const float2 s23 = __fadd2_rn(sum2[2], sum2[3]);
-            const float2 s03 = __fadd2_rn(s01, s23);
-            const float rs = s03.x + s03.y;
+            float f = 1.f;
             if (__any_sync(0xffffffffu, resc)) {
-                // O must hold P(i-1) V(i-1) before it is rescaled in place
+                // O must hold P(i-1) V(i-1) before it is rescaled in place, and the
+                // rescale must land before P(i) V(i) starts accumulating
                 if (!warp_wait(bars.pv_done(t), (i - 1) & 1, abort_flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const float f = resc ? ex2_approx(m_run - m_new) : 1.f;
+                f = resc ? ex2_approx(m_run - m_new) : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < PP_D / 32; ++c) {
                     float o[32];
@@ -361,13 +364,35 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                     tmem_st32(t_o + c * 32, o);
                 }
                 tmem_wait_st();
-                l_run *= f;
             }
-            l_run += rs;
-            m_run = m_new;
+            // pass 2: the second half is in registers; its P goes to columns 96-127
+            // (S columns already read) and is released to the tensor core at once;
+            // then the first half is read again and its P goes to columns 64-95
+            float2 sum2[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sum2[k] = make_float2(0.f, 0.f);
+            exp_half(s, sl2, m_new, sum2);
+            store_p_half(t_s + L::P_OFF + 32, s);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bars.p_full(t));  // P(i) and (rescaled) O ready
+            if (lane == 0) mbar_arrive(bars.p_half(t));  // P(i) of keys 64-127, (rescaled) O
+            tmem_ld32(t_s, s);
+            tmem_ld32(t_s + 32, s + 32);
+            tmem_wait_ld();
+            reg_fence32(s);
+            reg_fence32(s + 32);
+            exp_half(s, sl2, m_new, sum2);
+            store_p_half(t_s + L::P_OFF, s);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.p_full(t));  // all of P(i)
+            const float2 s01 = __fadd2_rn(sum2[0], sum2[1]);
+            const float2 s23 = __fadd2_rn(sum2[2], sum2[3]);
+            const float2 s03 = __fadd2_rn(s01, s23);
+            l_run = l_run * f + (s03.x + s03.y);
+            m_run = m_new;
         }
         if (ok && n > 0 && warp_wait(bars.pv_done(t), (n - 1) & 1, abort_flag, a.wait_ns)) {
             tc_fence_after();
