@@ -105,7 +105,8 @@ namespace {
 
 int sparse_attn(const void* q, const void* k, const void* v, const int32_t* idx, int topk, int B,
                 int H, int Nq, int Nk, int d, int T, float scale, void* o, float* lse,
-                int32_t* status, unsigned long long wait_ns, int skip_mma, void* stream) {
+                int32_t* status, unsigned long long wait_ns, int skip_mma, int force_pair,
+                void* stream) {
     if (!q || !k || !v || !o) return VELOX_EINVAL;
     if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || d < 1 || T < 1) return VELOX_EINVAL;
     if (!tile_ok(T) || !tile_ok(d)) return VELOX_EUNSUPPORTED;
@@ -135,6 +136,7 @@ int sparse_attn(const void* q, const void* k, const void* v, const int32_t* idx,
     a.status = status;
     a.wait_ns = wait_ns;
     a.skip_mma = skip_mma;
+    a.force_pair = force_pair;
     return velox::attn_fwd_launch(q, k, v, a, B, d, as_stream(stream));
 }
 
@@ -146,7 +148,7 @@ int velox_sparse_attn_fwd(const void* q, const void* k, const void* v, const int
                           int topk, int B, int H, int Nq, int Nk, int d, int T, float scale,
                           void* o, float* lse, int32_t* status, void* stream) {
     return sparse_attn(q, k, v, idx, topk, B, H, Nq, Nk, d, T, scale, o, lse, status,
-                       velox::WAIT_LIMIT_NS, 0, stream);
+                       velox::WAIT_LIMIT_NS, 0, 0, stream);
 }
 
 int velox_sparse_attn_fwd_test(const void* q, const void* k, const void* v, const int32_t* idx,
@@ -154,10 +156,11 @@ int velox_sparse_attn_fwd_test(const void* q, const void* k, const void* v, cons
                                void* o, float* lse, int32_t* status, double wait_limit_s,
                                int flags, void* stream) {
     if (!(wait_limit_s >= 1e-3 && wait_limit_s <= 10.0)) return VELOX_EINVAL;
-    if (flags & ~VELOX_TEST_SKIP_MMA) return VELOX_EINVAL;
+    if (flags & ~(VELOX_TEST_SKIP_MMA | VELOX_TEST_FORCE_PAIR)) return VELOX_EINVAL;
     return sparse_attn(q, k, v, idx, topk, B, H, Nq, Nk, d, T, scale, o, lse, status,
                        static_cast<unsigned long long>(wait_limit_s * 1e9),
-                       (flags & VELOX_TEST_SKIP_MMA) ? 1 : 0, stream);
+                       (flags & VELOX_TEST_SKIP_MMA) ? 1 : 0,
+                       (flags & VELOX_TEST_FORCE_PAIR) ? 1 : 0, stream);
 }
 
 size_t velox_kbar_cache_bytes(int B, int H, int max_past_chunks, int Nq, int d, int T) {

@@ -96,4 +96,10 @@ bool make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, 
 int attn_pp_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B,
                    cudaStream_t st);
 
+// The CTA-pair kernel (d = 128, T = 128) and the lists it takes.
+bool attn_pair_supported(const AttnArgs& a);
+bool attn_pair_preferred(const AttnArgs& a);
+int attn_pair_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B,
+                     cudaStream_t st);
+
 }  // namespace velox

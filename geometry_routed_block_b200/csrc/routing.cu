@@ -106,24 +106,50 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_q_kernel(const TIn* __restr
     if (threadIdx.x < D) qbar[blk * D + threadIdx.x] = out[threadIdx.x];
 }
 
-// One warp pools one [T][D] block: lane (cg, r0) reads 16-byte column group cg
-// of rows r0, r0 + RPW, ... (all its loads in flight at once, in batches),
+// Loads of one warp's [T][D] block: lane (cg, r0) reads 16-byte column group
+// cg of rows r0, r0 + RPW, ...; the first batch is issued by warp_pool_first so
+// that a caller can overlap it with other work.
+template <typename TIn, int D, int T>
+struct WarpPoolShape {
+    using V = VecTraits<TIn>;
+    static constexpr int TPR = D / V::VEC;
+    static constexpr int RPW = 32 / TPR;
+    static constexpr int LOADS = T / RPW;
+    static constexpr int BATCH = LOADS < 16 ? LOADS : 16;
+};
+
+template <typename TIn, int D, int T>
+__device__ __forceinline__ void warp_pool_first(const TIn* __restrict__ blk, int lane,
+                                                uint4* buf) {
+    using S = WarpPoolShape<TIn, D, T>;
+    const int cg = lane % S::TPR, r0 = lane / S::TPR;
+    const TIn* base = blk + static_cast<size_t>(r0) * D + cg * S::V::VEC;
+#pragma unroll
+    for (int i = 0; i < S::BATCH; ++i) buf[i] = ldg_stream(base + static_cast<size_t>(i) * S::RPW * D);
+}
+
+// One warp pools one [T][D] block: all of a lane's loads in flight at once, in
+// batches (the first batch already issued into `first` by warp_pool_first),
 // sums in fp32 pairs, then the lanes of a column group reduce by shuffles.
 // On return every lane holds the column sums of its group, times 1/T.
 template <typename TIn, int D, int T>
-__device__ __forceinline__ void warp_pool(const TIn* __restrict__ blk, int lane, float* kbar) {
+__device__ __forceinline__ void warp_pool_rest(const TIn* __restrict__ blk, int lane,
+                                               const uint4* first, float* kbar) {
     using V = VecTraits<TIn>;
-    constexpr int TPR = D / V::VEC;
-    constexpr int RPW = 32 / TPR;
-    constexpr int LOADS = T / RPW;
-    constexpr int BATCH = LOADS < 16 ? LOADS : 16;
+    using S = WarpPoolShape<TIn, D, T>;
+    constexpr int TPR = S::TPR;
+    constexpr int RPW = S::RPW;
+    constexpr int LOADS = S::LOADS;
+    constexpr int BATCH = S::BATCH;
     const int cg = lane % TPR, r0 = lane / TPR;
     const TIn* base = blk + static_cast<size_t>(r0) * D + cg * V::VEC;
     float acc[V::VEC];
 #pragma unroll
     for (int i = 0; i < V::VEC; ++i) acc[i] = 0.f;
 #pragma unroll
-    for (int b0 = 0; b0 < LOADS; b0 += BATCH) {
+    for (int i = 0; i < BATCH; ++i) V::add(acc, first[i]);
+#pragma unroll
+    for (int b0 = BATCH; b0 < LOADS; b0 += BATCH) {
         uint4 buf[BATCH];
 #pragma unroll
         for (int i = 0; i < BATCH; ++i)
@@ -138,6 +164,13 @@ __device__ __forceinline__ void warp_pool(const TIn* __restrict__ blk, int lane,
     }
 #pragma unroll
     for (int i = 0; i < V::VEC; ++i) kbar[i] = acc[i] * (1.0f / T);
+}
+
+template <typename TIn, int D, int T>
+__device__ __forceinline__ void warp_pool(const TIn* __restrict__ blk, int lane, float* kbar) {
+    uint4 first[WarpPoolShape<TIn, D, T>::BATCH];
+    warp_pool_first<TIn, D, T>(blk, lane, first);
+    warp_pool_rest<TIn, D, T>(blk, lane, first, kbar);
 }
 
 // CTA = one (b, h) slice of the grid; each warp walks its own past key blocks
@@ -156,16 +189,25 @@ __global__ void __launch_bounds__(POOL_THREADS)
 
     const int bh = blockIdx.y;
     const int t = threadIdx.x;
-    for (int i = t; i < r.m * D; i += POOL_THREADS) q_s[i] = qbar[static_cast<size_t>(bh) * r.m * D + i];
-    __syncthreads();
-
     const TIn* kh = k + static_cast<size_t>(bh) * r.Nk * D;
     const int warp = t >> 5, lane = t & 31;
     const int cg = lane % TPR, r0 = lane / TPR;
+    const int stride = gridDim.x * WARPS;
+    int kb = blockIdx.x * WARPS + warp;
+    // the first loads of this warp's first key block fly while q-bar is staged
+    uint4 first[WarpPoolShape<TIn, D, T>::BATCH];
+    if (kb < r.n_past)
+        warp_pool_first<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, first);
+    for (int i = t; i < r.m * D; i += POOL_THREADS) q_s[i] = qbar[static_cast<size_t>(bh) * r.m * D + i];
+    __syncthreads();
+
     float* srow = r.scores + static_cast<size_t>(bh) * r.m * r.n_past;
-    for (int kb = blockIdx.x * WARPS + warp; kb < r.n_past; kb += gridDim.x * WARPS) {
+    for (bool head = true; kb < r.n_past; kb += stride, head = false) {
         float kv[V::VEC];
-        warp_pool<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, kv);
+        if (head)
+            warp_pool_rest<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, first, kv);
+        else
+            warp_pool<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, kv);
         // every lane runs the same number of iterations (full-warp shuffles)
         for (int q0 = 0; q0 < r.m; q0 += RPW) {
             const int qb = q0 + r0;

@@ -27,6 +27,7 @@ struct AttnArgs {
     long long q_rows;        // B * H * Nq
     unsigned long long wait_ns;  // limit of every bounded wait
     int skip_mma;                // test hook: the tensor-core issuer issues nothing
+    int force_pair;              // test hook: d = T = 128 on the CTA-pair kernel
 };
 
 int attn_fwd_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B, int d,

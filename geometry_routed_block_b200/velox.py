@@ -28,6 +28,7 @@ VELOX_EBOUNDS = -5
 VELOX_STATUS_BAD_INDEX = 1
 VELOX_STATUS_TIMEOUT = 2
 VELOX_TEST_SKIP_MMA = 1
+VELOX_TEST_FORCE_PAIR = 2
 VELOX_BF16 = 0
 VELOX_F32 = 1
 CAM_FLOATS = 18
@@ -284,9 +285,10 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torc
 def sparse_attn_fwd_test(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                          idx: torch.Tensor | None, T: int, status: torch.Tensor,
                          wait_limit_s: float, flags: int, out: torch.Tensor | None = None,
-                         stream=None) -> torch.Tensor:
+                         lse: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """sparse_attn_fwd through the test entry point (bounded-wait limit and
-    failure-injection flags); returns O (unwritten when the waits ran out)."""
+    test-hook flags); returns O (unwritten when the waits ran out). An `lse`
+    tensor [B,H,Nq] f32, when given, receives the log-sum-exp."""
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -299,7 +301,7 @@ def sparse_attn_fwd_test(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if out is None:
         out = torch.empty_like(q)
     _check(lib.velox_sparse_attn_fwd_test(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), topk, B, H, Nq, Nk,
-                                          d, T, float(1.0 / math.sqrt(d)), _ptr(out), None,
+                                          d, T, float(1.0 / math.sqrt(d)), _ptr(out), _ptr(lse),
                                           _ptr(status), float(wait_limit_s), int(flags),
                                           _stream(stream)), "velox_sparse_attn_fwd_test")
     return out

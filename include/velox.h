@@ -184,6 +184,7 @@ VELOX_API int velox_sparse_attn_fwd(const void* q, const void* k, const void* v,
 
 /* test-hook flags of velox_sparse_attn_fwd_test */
 #define VELOX_TEST_SKIP_MMA 1
+#define VELOX_TEST_FORCE_PAIR 2
 
 /*
  * velox_sparse_attn_fwd with two test hooks for its failure path; not a step
@@ -197,7 +198,12 @@ VELOX_API int velox_sparse_attn_fwd(const void* q, const void* k, const void* v,
  *   flags         VELOX_TEST_SKIP_MMA: the tensor-core issuer issues nothing,
  *                 so no MMA completion ever arrives and the waits on them run
  *                 out (no MMA is in flight when tensor memory is freed); the
- *                 output is left unwritten. 0: a normal call.
+ *                 output is left unwritten.
+ *                 VELOX_TEST_FORCE_PAIR: for d = T = 128, run the CTA-pair
+ *                 kernel (two SMs per MMA, the union of two blocks' lists
+ *                 walked once) also for routed lists, which otherwise go to the
+ *                 single-SM two-block kernel; lists of more than 2048 blocks
+ *                 still go there. 0: a normal call.
  * Other arguments, results and errors are those of velox_sparse_attn_fwd;
  * VELOX_EINVAL also for a limit outside the range or an unknown flag.
  */
