@@ -4,7 +4,12 @@
 // "Tiefenanalyse" -- the router decides at the granularity of the kernel's
 // tile, so the kernel really skips the key blocks it is not given. Here one
 // CTA owns a 128-row query tile of one (batch, head) and walks only the key
-// blocks listed for its query block.
+// blocks listed for it. With 128-token blocks the tile is one query block.
+// With 64-token blocks it is two adjacent query blocks, which walk the union
+// of their two routed lists (adjacent blocks keep almost the same key blocks),
+// each entry tagged with which of the two listed it: the softmax warps of the
+// block that did not list a tile turn its S into P = 0, so each block attends
+// exactly to its own list and no MMA row is padding.
 //
 // CTA = 7 warps:
 //   warps 0-3  softmax / correction / epilogue; thread i owns query row i,
@@ -44,15 +49,21 @@ constexpr int WARP_TMA_K = 4;
 constexpr int WARP_MMA = 5;
 constexpr int WARP_TMA_V = 6;
 
+constexpr int WALK_MAX = 8192;           // walk entries: two lists of up to 4096 blocks
+constexpr int WALK_BITMAP_WORDS = 512;   // key blocks <= 16384 take the union by bitmap
+
 template <int D, int BN>
 struct Layout {
+    static constexpr bool PAIR = BN == 64;  // two 64-token query blocks per 128-row tile
     static constexpr int KV_TILE = BN * D * 2;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + KST * KV_TILE;
-    static constexpr int OFF_BAR = OFF_V + VST * KV_TILE;
+    static constexpr int OFF_WALK = OFF_V + VST * KV_TILE;  // int32 [WALK_MAX] (PAIR only)
+    static constexpr int OFF_BITMAP = OFF_WALK + (PAIR ? WALK_MAX * 4 : 0);  // uint32 [2][WORDS]
+    static constexpr int OFF_BAR = OFF_BITMAP + (PAIR ? 2 * WALK_BITMAP_WORDS * 4 : 0);
     // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2], pv_done[2]
     static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, walk length
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
     // tensor memory columns: S[2] (fp32; P_j, as bf16 pairs, overwrites the
@@ -91,13 +102,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int qb = blockIdx.x;
+    // first query block of the tile, and how many the tile holds (1 or 2)
+    const bool pair = L::PAIR && a.pair_tiles;
+    const int qb = pair ? 2 * blockIdx.x : blockIdx.x;
+    const int nblk = pair ? min(2, a.m - qb) : 1;
     const int bh = blockIdx.z * a.H + blockIdx.y;
-    const int n = a.n_sel;
 
     Bars bars{sbase + L::OFF_BAR};
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    int* walk_len = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);
+    const int* walk = reinterpret_cast<const int*>(smem + L::OFF_WALK);
+    const bool use_walk = pair && a.idx != nullptr;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -125,10 +141,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
     }
+    if (use_walk && warp == WARP_TMA_V) {
+        const int len = build_walk<WALK_BITMAP_WORDS>(
+            a, bh, qb, nblk > 1, reinterpret_cast<uint32_t*>(smem + L::OFF_BITMAP),
+            reinterpret_cast<int*>(smem + L::OFF_WALK), lane);
+        if (lane == 0) *walk_len = len;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int n = use_walk ? *walk_len : a.n_sel;
+    // which of the tile's blocks listed entry j (bit g: block qb + g)
+    auto listed = [&](int j) -> int {
+        if (use_walk) return walk[j] >> 16;
+        return pair ? (1 << nblk) - 1 : 1;
+    };
 
     if (warp == WARP_TMA_K || warp == WARP_TMA_V) {
         // ------------------------------------------------------------ producers
@@ -143,9 +171,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             auto empty = [&](int st) { return is_v ? bars.v_empty(st) : bars.k_empty(st); };
             const int krow0 = bh * a.Nk;
             const int32_t* row_idx =
-                a.idx ? a.idx + (static_cast<size_t>(bh) * a.m + qb) * static_cast<size_t>(n)
+                a.idx ? a.idx + (static_cast<size_t>(bh) * a.m + qb) * static_cast<size_t>(a.n_sel)
                       : nullptr;
             auto fetch = [&](int j) -> int {
+                if (use_walk) return walk[j] & 0xFFFF;  // validated when it was built
                 int kb = row_idx ? __ldg(row_idx + j) : j;
                 if (kb < 0 || kb >= a.n_kb) {
                     if (a.status && !is_v) atomicOr(a.status, VELOX_STATUS_BAD_INDEX);
@@ -231,6 +260,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         const uint32_t t_o = tmem + lane_base + L::TMEM_O;
         const float sl2 = a.scale_log2;
+        // the tile row's block: rows 0-63 are block qb, rows 64-127 block qb + 1
+        const int mybit = pair ? 1 << (warp >> 1) : 1;
         float m_run = -INFINITY;
         float l_run = 0.f;
         bool ok = true;
@@ -269,6 +300,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 break;
             }
             tc_fence_after();
+            if (!(listed(j) & mybit)) {
+                // a tile of the walk this warp's block did not list: P = 0
+                float z[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) z[k] = 0.f;
+                const uint32_t t_p = tmem + lane_base + L::TMEM_S + bi * BN;
+#pragma unroll
+                for (int c = 0; c < BN / 64; ++c) tmem_st32(t_p + c * 32, z);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars.p_full(bi));
+                continue;
+            }
             float s[BN];
             const uint32_t t_s = tmem + lane_base + L::TMEM_S + bi * BN;
             // first half of the row, then the second half in flight while the
@@ -296,7 +341,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             bool resc = false;
             if (mx > m_run + RESCALE_THRESHOLD) {
                 m_new = mx;
-                resc = (j > 0);
+                // O is still exactly 0 before the first tile this row's block listed
+                resc = m_run > -INFINITY;
             }
             // p = 2^(s * scale * log2e - m), two lanes of fp32 per FFMA2 / FADD2;
             // the pairs selected by EXP2_EMU_MASK run on the FMA pipe, the rest
@@ -365,7 +411,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (ok && n > 0 && warp_wait(bars.pv_done((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, a.wait_ns)) {
             tc_fence_after();
             const float inv = 1.f / l_run;
-            const bool store = row < a.T;
+            const bool store = row < nblk * a.T;
             const size_t grow = static_cast<size_t>(bh) * a.Nq + static_cast<size_t>(qb) * a.T + row;
             __nv_bfloat16* orow = a.o + grow * D;
 #pragma unroll 1
@@ -410,11 +456,13 @@ int launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B
     AttnArgs args = a;
     args.q = static_cast<const __nv_bfloat16*>(q);
     args.q_rows = static_cast<long long>(bh) * a.Nq;
+    // 64-token blocks: two per tile, unless a walk of two lists would not fit
+    args.pair_tiles = L::PAIR && (a.idx == nullptr || (a.n_sel <= WALK_MAX / 2 && a.n_kb <= 65535));
     auto kern = attn_fwd_kernel<D, BN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) !=
         cudaSuccess)
         return VELOX_ECUDA;
-    dim3 grid(a.m, a.H, B);
+    dim3 grid(args.pair_tiles ? (a.m + 1) / 2 : a.m, a.H, B);
     kern<<<grid, NTHREADS, L::SMEM, st>>>(tk, tv, args);
     return cudaGetLastError() == cudaSuccess ? VELOX_OK : VELOX_ECUDA;
 }

@@ -87,6 +87,84 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
     return true;
 }
 
+// The walk of two adjacent query blocks, built by one warp: the union of the
+// routed lists of query blocks qb0 and (if present) qb0 + 1, ascending, entry
+// = kb | (mask << 16) with bit g of mask set when list g holds kb (bm: scratch
+// bitmaps of 2 x WORDS words, so up to 32 * WORDS key blocks). A list that
+// repeats a block, or more key blocks than the bitmap holds, gives the
+// concatenation of the lists instead (masks one-hot), which keeps every listed
+// block, repeats included. Indices out of range are replaced by block 0 and
+// flagged in the status word. The same rows always give the same walk.
+// Returns its length (at most twice the list length).
+template <int WORDS>
+__device__ int build_walk(const AttnArgs& a, int bh, int qb0, bool has1, uint32_t* bm, int* out,
+                          int lane) {
+    const unsigned FULL = 0xffffffffu;
+    const int n = a.n_sel;
+    const int32_t* r0 = a.idx + (static_cast<size_t>(bh) * a.m + qb0) * static_cast<size_t>(n);
+    const int nlist = has1 ? 2 : 1;
+    const int nw = (a.n_kb + 31) >> 5;
+    bool bitmap = nw <= WORDS;
+    bool bad = false;
+    if (bitmap) {
+        for (int w = lane; w < 2 * WORDS; w += 32) bm[w] = 0;
+        __syncwarp();
+        bool dup = false;
+        for (int g = 0; g < nlist; ++g) {
+            const int32_t* row = r0 + static_cast<size_t>(g) * n;
+            for (int j = lane; j < n; j += 32) {
+                int kb = __ldg(row + j);
+                if (kb < 0 || kb >= a.n_kb) {
+                    bad = true;
+                    kb = 0;
+                }
+                const uint32_t bit = 1u << (kb & 31);
+                const uint32_t old = atomicOr(&bm[g * WORDS + (kb >> 5)], bit);
+                dup |= (old & bit) != 0;
+            }
+        }
+        __syncwarp();
+        bitmap = !__any_sync(FULL, dup);
+    }
+    if (__any_sync(FULL, bad) && lane == 0 && a.status) atomicOr(a.status, VELOX_STATUS_BAD_INDEX);
+    if (bitmap) {
+        constexpr int PER = WORDS / 32;  // words per lane
+        const int w0 = lane * PER;
+        int cnt = 0;
+#pragma unroll
+        for (int w = w0; w < w0 + PER; ++w)
+            if (w < nw) cnt += __popc(bm[w] | bm[WORDS + w]);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(FULL, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int pos = incl - cnt;
+        const int total = __shfl_sync(FULL, incl, 31);
+        for (int w = w0; w < w0 + PER && w < nw; ++w) {
+            const uint32_t u0 = bm[w], u1 = bm[WORDS + w];
+            uint32_t u = u0 | u1;
+            while (u) {
+                const int b = __ffs(u) - 1;
+                u &= u - 1;
+                const int mask = static_cast<int>(((u0 >> b) & 1u) | (((u1 >> b) & 1u) << 1));
+                out[pos++] = (w * 32 + b) | (mask << 16);
+            }
+        }
+        return total;
+    }
+    for (int g = 0; g < nlist; ++g) {
+        const int32_t* row = r0 + static_cast<size_t>(g) * n;
+        for (int j = lane; j < n; j += 32) {
+            int kb = __ldg(row + j);
+            if (kb < 0 || kb >= a.n_kb) kb = 0;
+            out[g * n + j] = kb | ((1 << g) << 16);
+        }
+    }
+    return nlist * n;
+}
+
 }  // namespace
 
 // rows x cols bf16 matrix (row-major), boxes of box_rows x 64 columns, 128-byte swizzle

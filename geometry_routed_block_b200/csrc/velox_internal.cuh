@@ -28,6 +28,7 @@ struct AttnArgs {
     unsigned long long wait_ns;  // limit of every bounded wait
     int skip_mma;                // test hook: the tensor-core issuer issues nothing
     int force_pair;              // test hook: d = T = 128 on the CTA-pair kernel
+    int pair_tiles;              // set by the launcher: two 64-token blocks per 128-row tile
 };
 
 int attn_fwd_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B, int d,

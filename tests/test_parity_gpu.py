@@ -530,3 +530,45 @@ def test_cached_routing_equals_streaming_routing(vx, cfg):
     # no past chunk yet: only the current chunk's blocks
     only = vx.route_topk_cached(q, kbar, 0, None, s.alpha, s.m, s.T).cpu().numpy()
     assert (only == np.arange(s.m)).all()
+
+
+# ---------------------------------------------------------------- 64-token blocks
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_t64_routed_attention_pairs_blocks(vx, d):
+    """64-token blocks (workload 4's generator at P = 8 with T = 64): the kernel
+    packs two adjacent query blocks into one 128-row tile that walks the union
+    of their routed lists; every query block of two heads against the oracle,
+    on the oracle's selection, and the GPU selection against the oracle's."""
+    heads = (2, 19)
+    c = synth.make_case(4, P=8, heads=heads, T=64, d=d)
+    s = c.shape
+    assert s.T == 64 and s.m == 72
+    sl = vo.slices_build(c.past_depth[0], c.past_poses[0], c.past_intr[0])
+    counts = vo.block_overlap(c.cur_depth, c.cur_cam, sl[None], s.F, s.T)
+    q, k, v = c.q[0], c.k[0], c.v[0]
+    want, s_mod = oracle_route_per_head(q, k, counts, s.alpha, s.topk, s.T)
+    idx = vx.route_topk(dev(q), dev(k), dev(counts), s.alpha, s.topk, s.T)
+    ties = compare_selection(idx.cpu().numpy(), want, s_mod, s.m,
+                             label=f"workload 4, P = 8, T = 64, d = {d}, heads {heads}")
+    assert ties <= tie_bound(2 * s.m)
+    rows = [(0, i, qb) for i in range(2) for qb in range(s.m)]
+    attention_rows_vs_oracle(vx, q, k, v, want, s.T, rows,
+                             label=f"workload 4, P = 8, T = 64, d = {d} (paired query blocks)")
+
+
+def test_t64_long_lists_fall_back_to_one_block_per_tile(vx):
+    """A routed list longer than two of them fit in the tile's walk (4,096
+    blocks): one 64-token block per tile, still exact against the oracle."""
+    rng = np.random.default_rng(64)
+    T, d, B, H, m, nkb, topk = 64, 128, 1, 1, 3, 4500, 4200
+    f = lambda *sh: synth.f32_to_bf16_bits(rng.standard_normal(sh, dtype=np.float32))
+    q, k, v = f(B, H, m * T, d), f(B, H, nkb * T, d), f(B, H, nkb * T, d)
+    idx = np.stack([np.sort(rng.choice(nkb, topk, replace=False)) for _ in range(m)])
+    idx = idx.reshape(B, H, m, topk).astype(np.int32)
+    o, lse = vx.sparse_attn_fwd(dev(q), dev(k), dev(v), dev(idx), T)
+    ref = vo.sparse_attention(q, k, v, idx, T, rows=[(0, 0, qb) for qb in range(m)])
+    for (b, h, qb), (o_ref, lse_ref) in ref.items():
+        sl_ = slice(qb * T, (qb + 1) * T)
+        compare_attention(o[b, h, sl_], o_ref, f"T = 64, 4,200-block list, row {qb}")
+        assert np.abs(lse[b, h, sl_].cpu().numpy() - lse_ref).max() < 1e-3
