@@ -66,9 +66,9 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # launch at the headline workload, from a one-pass ncu capture of this kernel at full
 # size; reported only while the kernel sources still hash to what was captured.
 ATTN_TRAFFIC = {
-    "bytes_per_launch": 642.18e6 + 22.82e6,
-    "sources": {"attention_pp.cu": "13e4340e74204946", "attn_common.cuh": "edbf6bcdb3a2cde6",
-                "ptx.cuh": "34475d094993081f"},
+    "bytes_per_launch": 642.73e6 + 23.11e6,
+    "sources": {"attention_pp.cu": "b928acde795e1f93", "attn_common.cuh": "eb65731a5f58689c",
+                "ptx.cuh": "16d190c725154d53"},
 }
 
 
@@ -415,13 +415,15 @@ def time_loop(torch, fn, reps):
 SWEEP_P = (8, 16, 24, 32, 96)
 
 
-def sweep_point(torch, vx, device, P: int, reps: int, peaks: dict, status):
+def sweep_point(torch, vx, device, P: int, reps: int, peaks: dict, status, T: int = 128,
+                d: int = 128):
     """Workload 4 at P past chunks on this GPU (geometry from the synthetic
-    trajectory, Q/K/V drawn on the device with workload 3's structure): routing,
-    sparse attention and dense attention timed alone with CUDA events. Returns
-    the record and, for the oracle check, head 0's inputs and selection."""
+    trajectory, Q/K/V drawn on the device with workload 3's structure; other
+    block sizes T and head dims d on request): routing, sparse attention and
+    dense attention timed alone with CUDA events. Returns the record and, for
+    the oracle check, head 0's inputs and selection."""
     geo = synth.geometry_only(4, P=P)
-    s = synth.shape_for(4, P=P)
+    s = synth.shape_for(4, P=P, T=T, d=d)
     q, k, v = draw_qkv_on_device(torch, s, geo.meta["view_overlap"], 1004 + P, device)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
     slices = vx.slices_build(dev(geo.past_depth[0]), dev(geo.past_poses[0]), dev(geo.past_intr[0]))
@@ -445,7 +447,8 @@ def sweep_point(torch, vx, device, P: int, reps: int, peaks: dict, status):
     attn_tf = kf / (t_attn * 1e-3) / 1e12
     route_gbs = rbytes / (t_route * 1e-3) / 1e9
     rec = {
-        "P": P, "key_blocks": s.nKB, "topk": s.topk, "kept_fraction": round(s.topk / s.nKB, 4),
+        "P": P, "T": s.T, "d": s.d, "key_blocks": s.nKB, "topk": s.topk,
+        "kept_fraction": round(s.topk / s.nKB, 4),
         "routing_ms": round(t_route, 4), "routing_gbs": round(route_gbs, 1),
         "routing_hbm_frac": round(route_gbs / peaks["hbm_gbs"], 4),
         "sparse_attn_ms": round(t_attn, 4), "attn_tflops_kept": round(attn_tf, 1),
@@ -748,6 +751,14 @@ def run_gpu(args):
             checks.append(chk)
             torch.cuda.empty_cache()
         out["sweep"] = sweep
+        # the other block sizes and head dims the kernels support, at chunk 48
+        shapes = []
+        for T, d in ((64, 128), (64, 64), (128, 64)):
+            rec, _ = sweep_point(torch, vx, device, 48, max(3, min(10, args.steps // 20)), peaks,
+                                 w.status, T=T, d=d)
+            shapes.append(rec)
+            torch.cuda.empty_cache()
+        out["tile_shapes"] = shapes
         pipe = pipeline_measure(torch, vx, device, layers=30, steps=3, warmup=3, seed=1005)
         out["pipeline"] = {key: pipe[key] for key in (
             "layers", "ms_per_step", "tflops_kept", "geometry_ms", "geometry_done_after_ms",
