@@ -99,6 +99,9 @@ __device__ __forceinline__ void pool_block(const TIn* __restrict__ src, float* o
 template <typename TIn, int D, int T>
 __global__ void __launch_bounds__(POOL_THREADS) pool_q_kernel(const TIn* __restrict__ q, float* qbar) {
     using V = VecTraits<TIn>;
+    // the scorer, launched as this grid's dependent, may start at once: it
+    // streams its first key blocks and waits for q-bar only when it needs it
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ float red[(POOL_THREADS / (D / V::VEC)) * D];
     __shared__ float out[D];
     const size_t blk = blockIdx.x;
@@ -198,6 +201,8 @@ __global__ void __launch_bounds__(POOL_THREADS)
     uint4 first[WarpPoolShape<TIn, D, T>::BATCH];
     if (kb < r.n_past)
         warp_pool_first<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, first);
+    // q-bar comes from the preceding pool_q grid (a no-op without a dependent launch)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int i = t; i < r.m * D; i += POOL_THREADS) q_s[i] = qbar[static_cast<size_t>(bh) * r.m * D + i];
     __syncthreads();
 
@@ -685,7 +690,19 @@ int route_typed(const TIn* q, const TIn* k, const RouteArgs& r, cudaStream_t st)
         const int gx_max = max(1, occ * sms / BH);
         const int per_warp = (r.n_past + warps * gx_max - 1) / (warps * gx_max);
         const int gx = max(1, (r.n_past + warps * per_warp - 1) / (warps * per_warp));
-        kern<<<dim3(gx, BH), POOL_THREADS, smem, st>>>(k, r.qbar, r);
+        // launched as pool_q's programmatic dependent (see pool_score_kernel)
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(gx, BH);
+        cfg.blockDim = dim3(POOL_THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, k, static_cast<const float*>(r.qbar), r) != cudaSuccess)
+            return VELOX_ECUDA;
         }
     }
     // the counts are read by the selection only: it may wait for them alone
