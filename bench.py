@@ -7,18 +7,22 @@ One step = one pass of the whole hot path over one chunk's synthetic inputs,
 with the KV cache resident in HBM: frustum slices of every past chunk, slice
 overlap counts, geometry-modulated top-k routing (pooling + scores + select)
 and block-sparse attention over the routed blocks. The slices and counts are
-built on a side stream while the keys are pooled (only the selection waits
-for them), as the method builds its slices asynchronously to denoising. `value` is the whole-job
-throughput in TFLOP/s of attention work on the kept blocks
+built on a side stream one step ahead: chunk n+1's are built while chunk n's
+attention runs (the selection of a step waits only for its own counts, built
+during the step before), as the method builds its slices asynchronously to
+denoising; the timed steps therefore hold one extra geometry pass (the next
+chunk's). `value` is the whole-job throughput in TFLOP/s of attention work on
+the kept blocks
 (4 * B * H * m * topk * T^2 * d per step) divided by the step time. The dense
 attention over every block (this library's own dense attention) is timed
 separately for the speedup.
 
-Multi-GPU (torchrun, one process per GPU): every rank runs its own chunk
-(seed + rank) -- heads/chunks are independent units, there is no data-path
-collective -- and the time is the max over ranks ("scaling": "weak"). With
---shard heads the ranks split the heads of one chunk instead, replicate the
-geometry and all-gather O every step ("scaling": "strong").
+Multi-GPU (torchrun, one process per GPU): by default the ranks split the 24
+heads of one chunk (routing and attention of a head read only that head's
+Q/K/V; the geometry is replicated) and all-gather O in place every step
+("scaling": "strong"); with --shard chunks every rank runs its own chunk
+(seed + rank) with no data-path collective ("scaling": "weak"). The time is the
+max over ranks.
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload (the oracle stands in for a reference
@@ -310,16 +314,24 @@ class Workload:
         self.side = torch.cuda.Stream(device=device)
         self.geo_ready = torch.cuda.Event()
         self.after_attend = None  # e.g. the all-gather of O when heads are sharded
+        # geometry one step ahead (step_ahead): double-buffered counts, with events
+        # for "counts j built" and "the selection reading counts j done"
+        self.counts2 = [self.counts, torch.empty_like(self.counts)]
+        self.geo_ev = [torch.cuda.Event(), torch.cuda.Event()]
+        self.sel_ev = [torch.cuda.Event(), torch.cuda.Event()]
+        self.cur = None
 
-    def geometry(self):
+    def geometry(self, counts=None, depth=None, cam=None):
         vx, s = self.vx, self.s
         vx.slices_build(self.past_depth, self.past_poses, self.past_intr, out=self.slices)
-        vx.block_overlap(self.cur_depth, self.cur_cam, self.slices[None], s.F, s.T, out=self.counts)
+        vx.block_overlap(self.cur_depth if depth is None else depth,
+                         self.cur_cam if cam is None else cam, self.slices[None], s.F, s.T,
+                         out=self.counts if counts is None else counts)
 
-    def route(self, ready=None):
+    def route(self, ready=None, counts=None):
         s = self.s
-        self.vx.route_topk(self.q, self.k, self.counts, s.alpha, s.topk, s.T, ws=self.ws,
-                           out=self.idx, counts_ready=ready)
+        self.vx.route_topk(self.q, self.k, self.counts if counts is None else counts, s.alpha,
+                           s.topk, s.T, ws=self.ws, out=self.idx, counts_ready=ready)
 
     def attend(self):
         self.vx.sparse_attn_fwd(self.q, self.k, self.v, self.idx, self.s.T, out=self.o,
@@ -353,6 +365,51 @@ class Workload:
         self.attend()
         if ev is not None:
             ev[3].record(main)
+
+    def prime(self, depth=None, cam=None, ready=None):
+        """Builds the first step's counts on the side stream (step_ahead's prologue)."""
+        torch = self.torch
+        self.side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(self.side):
+            if ready is not None:
+                self.side.wait_event(ready)
+            self.geometry(self.counts2[0], depth, cam)
+            self.geo_ev[0].record(self.side)
+        self.cur = 0
+
+    def step_ahead(self, ev=None, route=None, next_depth=None, next_cam=None, next_ready=None):
+        """One step with the geometry pipelined one step ahead: routing (its
+        selection waits for the counts built during the previous step), then
+        attention; the next step's slices and counts are built on the side stream
+        once this step's selection is done, so they run under this step's
+        attention instead of competing with the scorer for SMs (the method builds
+        slices asynchronously to denoising). next_depth / next_cam: the next
+        step's inputs (default: this step's), next_ready: an event they wait for.
+        ev: routing (ev0 -> ev2, including any wait for the counts) and
+        attention (ev2 -> ev3)."""
+        torch = self.torch
+        main = torch.cuda.current_stream()
+        if self.cur is None:
+            self.prime()
+        j = self.cur
+        if ev is not None:
+            ev[0].record(main)
+        (route or self.route)(ready=self.geo_ev[j], counts=self.counts2[j])
+        self.sel_ev[j].record(main)
+        if ev is not None:
+            ev[2].record(main)
+        # counts2[1 - j] was last read by the previous step's selection, which the
+        # stream order puts before this one
+        self.side.wait_event(self.sel_ev[j])
+        with torch.cuda.stream(self.side):
+            if next_ready is not None:
+                self.side.wait_event(next_ready)
+            self.geometry(self.counts2[1 - j], next_depth, next_cam)
+            self.geo_ev[1 - j].record(self.side)
+        self.attend()
+        if ev is not None:
+            ev[3].record(main)
+        self.cur = 1 - j
 
 
 def reduce_max(values, device=None):
@@ -504,7 +561,7 @@ def run_gpu(args):
 
     # warm-up (also the first-call costs: tensor-map encode, attribute set)
     for _ in range(max(3, args.warmup)):
-        w.step()
+        w.step_ahead()
     w.dense()
     torch.cuda.synchronize()
 
@@ -517,18 +574,20 @@ def run_gpu(args):
         t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t_start.record()
         for i in range(args.steps):
-            w.step(evs[i])
+            w.step_ahead(evs[i])
         t_end.record()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
     clocks = clk.summary()
     ms_total = t_start.elapsed_time(t_end)
-    geo_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     route_ms = statistics.mean(e[0].elapsed_time(e[2]) for e in evs)
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     status = int(w.status.item())
     gpu_idx = w.idx.cpu().numpy()
+    # the geometry (slices + overlap counts) alone; in the steps it runs on the side
+    # stream under the previous step's attention
+    geo_ms = time_loop(torch, w.geometry, 20)
 
     # ---- pooled-key cache: each past chunk's key blocks pooled once when the chunk
     # was appended; per step the routing reads the 21 MB cache instead of 1.36 GB of K
@@ -536,12 +595,12 @@ def run_gpu(args):
     append_ms = time_loop(torch, lambda: [w.vx.kbar_append(w.k, s.Nq, s.T, j, kbar)
                                           for j in range(s.P)], 3) / s.P
 
-    def route_cached(ready=None):
-        w.vx.route_topk_cached(w.q, kbar, s.P, w.counts, s.alpha, s.topk, s.T, ws=w.ws, out=w.idx,
-                               counts_ready=ready)
+    def route_cached(ready=None, counts=None):
+        w.vx.route_topk_cached(w.q, kbar, s.P, w.counts if counts is None else counts, s.alpha,
+                               s.topk, s.T, ws=w.ws, out=w.idx, counts_ready=ready)
 
     def step_cached():
-        w.step(route=route_cached)
+        w.step_ahead(route=route_cached)
 
     route_cached()
     route_cached_ms = time_loop(torch, route_cached, 20)
@@ -596,6 +655,9 @@ def run_gpu(args):
             consumed[b].record(compute)
             o_read[b].record(compute)
         upload(0)
+        # the first step's geometry from its uploaded depth and camera; every later
+        # step's is built during the step before it (step_ahead)
+        w.prime(stage[0]["depth"], stage[0]["cam"], uploaded[0])
         for i in range(n):
             b = i & 1
             if i + 1 < n:
@@ -606,7 +668,9 @@ def run_gpu(args):
             w.v[:, :, s.P * s.Nq:].copy_(stage[b]["v"])
             w.q, w.cur_depth, w.cur_cam, w.o = (stage[b]["q"], stage[b]["depth"], stage[b]["cam"],
                                                 stage[b]["o"])
-            w.step()
+            nxt = stage[b ^ 1] if i + 1 < n else stage[b]
+            w.step_ahead(next_depth=nxt["depth"], next_cam=nxt["cam"],
+                         next_ready=uploaded[b ^ 1] if i + 1 < n else None)
             consumed[b].record(compute)
             o_ready[b].record(compute)
             with torch.cuda.stream(down):
@@ -615,7 +679,9 @@ def run_gpu(args):
                 o_read[b].record(down)
         compute.wait_stream(down)
         compute.wait_stream(up)
+        compute.wait_stream(w.side)
         w.q, w.cur_depth, w.cur_cam, w.o = q0, depth0, cam0, o0
+        w.cur = None  # the next step primes its own geometry again
 
     e2e_reps = max(3, min(50, args.steps // 4))
     e2e_run(2)
