@@ -16,8 +16,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libvelox.so")
-SOURCES = ["api.cu", "attention.cu", "attention_pp.cu", "attention_pair.cu", "routing.cu",
-           "geometry.cu"]
+SOURCES = ["api.cu", "attention.cu", "attention_pp.cu", "attention_pair.cu", "attention_pp64.cu",
+           "routing.cu", "geometry.cu"]
 HEADERS = ["ptx.cuh", "velox_internal.cuh", "attn_common.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 

@@ -504,7 +504,9 @@ int attn_fwd_launch(const void* q, const void* k, const void* v, const AttnArgs&
         return (attn_pair_preferred(a) || (a.force_pair && attn_pair_supported(a)))
                    ? attn_pair_launch(q, k, v, a, B, st)
                    : attn_pp_launch(q, k, v, a, B, st);
-    if (d == 128 && a.T == 64) return launch<128, 64>(q, k, v, a, B, st);
+    if (d == 128 && a.T == 64)
+        return attn_pp64_supported(a) ? attn_pp64_launch(q, k, v, a, B, st)
+                                      : launch<128, 64>(q, k, v, a, B, st);
     if (d == 64 && a.T == 128) return launch<64, 128>(q, k, v, a, B, st);
     if (d == 64 && a.T == 64) return launch<64, 64>(q, k, v, a, B, st);
     return VELOX_EUNSUPPORTED;

@@ -89,15 +89,17 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
 
 // The walk of two adjacent query blocks, built by one warp: the union of the
 // routed lists of query blocks qb0 and (if present) qb0 + 1, ascending, entry
-// = kb | (mask << 16) with bit g of mask set when list g holds kb (bm: scratch
+// = kb | (mask << SHIFT) with bit g of mask set when list g holds kb (OutT and
+// SHIFT: int and 16, or a 16-bit entry with SHIFT 14 when every key block
+// index is below 2^14; bm: scratch
 // bitmaps of 2 x WORDS words, so up to 32 * WORDS key blocks). A list that
 // repeats a block, or more key blocks than the bitmap holds, gives the
 // concatenation of the lists instead (masks one-hot), which keeps every listed
 // block, repeats included. Indices out of range are replaced by block 0 and
 // flagged in the status word. The same rows always give the same walk.
 // Returns its length (at most twice the list length).
-template <int WORDS>
-__device__ int build_walk(const AttnArgs& a, int bh, int qb0, bool has1, uint32_t* bm, int* out,
+template <int WORDS, typename OutT = int, int SHIFT = 16>
+__device__ int build_walk(const AttnArgs& a, int bh, int qb0, bool has1, uint32_t* bm, OutT* out,
                           int lane) {
     const unsigned FULL = 0xffffffffu;
     const int n = a.n_sel;
@@ -149,7 +151,7 @@ __device__ int build_walk(const AttnArgs& a, int bh, int qb0, bool has1, uint32_
                 const int b = __ffs(u) - 1;
                 u &= u - 1;
                 const int mask = static_cast<int>(((u0 >> b) & 1u) | (((u1 >> b) & 1u) << 1));
-                out[pos++] = (w * 32 + b) | (mask << 16);
+                out[pos++] = static_cast<OutT>((w * 32 + b) | (mask << SHIFT));
             }
         }
         return total;
@@ -159,7 +161,7 @@ __device__ int build_walk(const AttnArgs& a, int bh, int qb0, bool has1, uint32_
         for (int j = lane; j < n; j += 32) {
             int kb = __ldg(row + j);
             if (kb < 0 || kb >= a.n_kb) kb = 0;
-            out[g * n + j] = kb | ((1 << g) << 16);
+            out[g * n + j] = static_cast<OutT>(kb | ((1 << g) << SHIFT));
         }
     }
     return nlist * n;
@@ -173,6 +175,12 @@ bool make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, 
 // The two-query-tile kernel (d = 128, T = 128); returns VELOX_* codes.
 int attn_pp_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B,
                    cudaStream_t st);
+
+// The two-query-tile kernel for 64-token blocks (d = 128): each tile is two
+// query blocks, each key tile two entries of their walk; the lists it takes.
+bool attn_pp64_supported(const AttnArgs& a);
+int attn_pp64_launch(const void* q, const void* k, const void* v, const AttnArgs& a, int B,
+                     cudaStream_t st);
 
 // The CTA-pair kernel (d = 128, T = 128) and the lists it takes.
 bool attn_pair_supported(const AttnArgs& a);
