@@ -1,7 +1,9 @@
 """The two-tile attention kernel for 64-token blocks (head dim 128): a CTA owns
 four query blocks as two 128-row tiles, each tile walking the union of its two
-blocks' routed lists, two walk entries per 128-key tile. Element by element
-against the oracle on what is particular to it: CTAs with one to four query
+blocks' routed lists, two walk entries per 128-key tile. (With head dim 64 the
+library keeps the one-tile kernel, which pairs two blocks per tile; the same
+cases run on it.) Element by element against the oracle on what is particular
+to the two-tile kernel: CTAs with one to four query
 blocks, adjacent blocks with disjoint lists (one block's rows see masked
 entries before its first listed one), identical lists, repeated blocks (the
 concatenated walk), odd walk lengths (a half tile no block listed), tiles whose
@@ -20,6 +22,7 @@ from tests.parity_utils import compare_attention, dev
 pytestmark = pytest.mark.gpu
 
 T, D = 64, 128
+DIMS = pytest.mark.parametrize("d", [128, 64])
 
 
 @pytest.fixture(scope="module")
@@ -28,9 +31,9 @@ def vx():
     return velox
 
 
-def _qkv(rng, B, H, m, nkb):
+def _qkv(rng, B, H, m, nkb, d=D):
     f = lambda *sh: synth.f32_to_bf16_bits(rng.standard_normal(sh, dtype=np.float32))
-    return f(B, H, m * T, D), f(B, H, nkb * T, D), f(B, H, nkb * T, D)
+    return f(B, H, m * T, d), f(B, H, nkb * T, d), f(B, H, nkb * T, d)
 
 
 def _check(vx, q, k, v, idx, label, rows=None, lse_tol=1e-3):
@@ -51,20 +54,23 @@ def _check(vx, q, k, v, idx, label, rows=None, lse_tol=1e-3):
         assert np.abs(lse[b, h, sl].cpu().numpy() - lse_ref).max() < lse_tol, label
 
 
+@DIMS
 @pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 6, 7, 9])
-def test_ragged_ctas_random_lists(vx, m):
-    rng = np.random.default_rng(640 + m)
+def test_ragged_ctas_random_lists(vx, m, d):
+    rng = np.random.default_rng(640 + m + d)
     B, H, nkb, topk = 2, 3, 23, 6
-    q, k, v = _qkv(rng, B, H, m, nkb)
+    q, k, v = _qkv(rng, B, H, m, nkb, d)
     idx = np.stack([rng.choice(nkb, topk, replace=False) for _ in range(B * H * m)])
-    _check(vx, q, k, v, idx.reshape(B, H, m, topk).astype(np.int32), f"m = {m}, shuffled lists")
+    _check(vx, q, k, v, idx.reshape(B, H, m, topk).astype(np.int32),
+           f"m = {m}, d = {d}, shuffled lists")
 
 
+@DIMS
 @pytest.mark.parametrize("kind", ["disjoint", "identical", "repeats", "nested"])
-def test_list_structures(vx, kind):
+def test_list_structures(vx, kind, d):
     rng = np.random.default_rng({"disjoint": 1, "identical": 2, "repeats": 3, "nested": 4}[kind])
     B, H, m, nkb, topk = 1, 2, 8, 40, 9
-    q, k, v = _qkv(rng, B, H, m, nkb)
+    q, k, v = _qkv(rng, B, H, m, nkb, d)
     idx = np.empty((B, H, m, topk), dtype=np.int32)
     for h in range(H):
         for qb in range(m):
@@ -90,34 +96,37 @@ def test_list_structures(vx, kind):
                     pad = rng.choice(np.setdiff1d(np.arange(nkb), idx[0, h, qb - 1]),
                                      topk - len(sub), replace=False)
                     idx[0, h, qb] = np.concatenate([sub, pad])
-    _check(vx, q, k, v, idx, f"{kind} lists")
+    _check(vx, q, k, v, idx, f"{kind} lists, d = {d}")
 
 
+@DIMS
 @pytest.mark.parametrize("nkb", [1, 2, 11, 64])
-def test_dense_walks(vx, nkb):
-    rng = np.random.default_rng(6400 + nkb)
-    q, k, v = _qkv(rng, 1, 2, 6, nkb)
-    _check(vx, q, k, v, None, f"dense over {nkb} key blocks")
+def test_dense_walks(vx, nkb, d):
+    rng = np.random.default_rng(6400 + nkb + d)
+    q, k, v = _qkv(rng, 1, 2, 6, nkb, d)
+    _check(vx, q, k, v, None, f"dense over {nkb} key blocks, d = {d}")
 
 
-def test_large_logits_rescale(vx):
-    rng = np.random.default_rng(6464)
+@DIMS
+def test_large_logits_rescale(vx, d):
+    rng = np.random.default_rng(6464 + d)
     B, H, m, nkb = 1, 2, 6, 40
-    qf = rng.standard_normal((B, H, m * T, D), dtype=np.float32)
-    kf = rng.standard_normal((B, H, nkb * T, D), dtype=np.float32)
+    qf = rng.standard_normal((B, H, m * T, d), dtype=np.float32)
+    kf = rng.standard_normal((B, H, nkb * T, d), dtype=np.float32)
     ramp = np.linspace(0.2, 6.0, nkb * T, dtype=np.float32)[None, None, :, None]
     kf = kf * ramp + ramp * qf.mean(axis=2, keepdims=True)
     q, k = synth.f32_to_bf16_bits(qf), synth.f32_to_bf16_bits(kf)
-    v = synth.f32_to_bf16_bits(rng.standard_normal((B, H, nkb * T, D), dtype=np.float32))
+    v = synth.f32_to_bf16_bits(rng.standard_normal((B, H, nkb * T, d), dtype=np.float32))
     idx = np.stack([np.sort(rng.choice(nkb, 17, replace=False)) for _ in range(B * H * m)])
     _check(vx, q, k, v, idx.reshape(B, H, m, 17).astype(np.int32), "rescale, routed",
            lse_tol=2e-3)
     _check(vx, q, k, v, None, "rescale, dense", lse_tol=2e-3)
 
 
-def test_bad_indices_flagged(vx):
-    rng = np.random.default_rng(646)
-    q, k, v = _qkv(rng, 1, 1, 5, 16)
+@DIMS
+def test_bad_indices_flagged(vx, d):
+    rng = np.random.default_rng(646 + d)
+    q, k, v = _qkv(rng, 1, 1, 5, 16, d)
     idx = np.array([[[[0, 1, -5], [2, 16, 3], [4, 5, 6], [7, 8, 99], [1, 2, 3]]]], dtype=np.int32)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o, _ = vx.sparse_attn_fwd(dev(q), dev(k), dev(v), dev(idx), T, status=status)
