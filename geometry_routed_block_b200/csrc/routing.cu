@@ -201,6 +201,9 @@ __global__ void __launch_bounds__(POOL_THREADS)
     uint4 first[WarpPoolShape<TIn, D, T>::BATCH];
     if (kb < r.n_past)
         warp_pool_first<TIn, D, T>(kh + static_cast<size_t>(kb) * T * D, lane, first);
+    // the selection, launched as this grid's dependent, may be scheduled now:
+    // it waits for this grid to finish before it reads a score
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // q-bar comes from the preceding pool_q grid (a no-op without a dependent launch)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int i = t; i < r.m * D; i += POOL_THREADS) q_s[i] = qbar[static_cast<size_t>(bh) * r.m * D + i];
@@ -281,6 +284,8 @@ __global__ void __launch_bounds__(256) score_cached_kernel(const float* __restri
     constexpr int KP = D + 4;          // padded row: 16-byte aligned, 128-bit reads conflict-free
     float* q_s = sm;                   // [m][D]
     float* k_s = q_s + r.m * D;        // [SC_KT][KP]
+    // the selection, launched as this grid's dependent, may be scheduled now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int bh = blockIdx.y;
     const int kb0 = blockIdx.x * SC_KT;
     const int nk = min(SC_KT, r.n_past - kb0);
@@ -409,6 +414,8 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_kernel(const SelArgs a)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * SEL_WARPS + warp;
     if (row >= a.rows) return;
+    // launched as the scorer's dependent: scores (and counts) only after it is done
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int n_past = a.n_past, m = a.m, k_past = a.k_past;
     const float* sc = a.scores + static_cast<size_t>(row) * n_past;
     int32_t* out = a.idx + static_cast<size_t>(row) * a.topk;
@@ -515,6 +522,8 @@ __global__ void __launch_bounds__(THREADS) select_cta_kernel(const SelArgs a) {
         for (int i = t; i < n_past; i += THREADS) out[i] = i;
         return;
     }
+    // launched as the scorer's dependent: scores (and counts) only after it is done
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     RowMod mod{nullptr, a.alpha, a.invT, 1.0f / static_cast<float>(a.m)};
     if (warp == 0) {
         const RowMod w = row_mod(a, row, lane);
@@ -634,23 +643,45 @@ __global__ void __launch_bounds__(THREADS) select_cta_kernel(const SelArgs a) {
     }
 }
 
+// A kernel launched as the programmatic dependent of the one before it in the
+// stream: its CTAs may be scheduled while that grid still runs, and wait for it
+// with griddepcontrol.wait before they read what it writes.
+template <typename Kern, typename... Args>
+cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             const Args&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// the selection, launched as the dependent of the scorer
 int select_launch(const SelArgs& a, cudaStream_t st) {
     constexpr int TH = SEL_CTA_THREADS;
     const size_t smem = static_cast<size_t>(a.n_past) * sizeof(uint32_t);
     const dim3 grid(a.rows), block(TH);
+    cudaError_t e;
     if (a.n_past <= TH * 1)
-        select_cta_kernel<TH, 1><<<grid, block, smem, st>>>(a);
+        e = launch_dependent(select_cta_kernel<TH, 1>, grid, block, smem, st, a);
     else if (a.n_past <= TH * 2)
-        select_cta_kernel<TH, 2><<<grid, block, smem, st>>>(a);
+        e = launch_dependent(select_cta_kernel<TH, 2>, grid, block, smem, st, a);
     else if (a.n_past <= TH * 4)
-        select_cta_kernel<TH, 4><<<grid, block, smem, st>>>(a);
+        e = launch_dependent(select_cta_kernel<TH, 4>, grid, block, smem, st, a);
     else if (a.n_past <= TH * 8)
-        select_cta_kernel<TH, 8><<<grid, block, smem, st>>>(a);
+        e = launch_dependent(select_cta_kernel<TH, 8>, grid, block, smem, st, a);
     else if (a.n_past <= TH * 16)
-        select_cta_kernel<TH, 16><<<grid, block, smem, st>>>(a);
+        e = launch_dependent(select_cta_kernel<TH, 16>, grid, block, smem, st, a);
     else
-        select_kernel<<<(a.rows + SEL_WARPS - 1) / SEL_WARPS, SEL_WARPS * 32, 0, st>>>(a);
-    return VELOX_OK;
+        e = launch_dependent(select_kernel, dim3((a.rows + SEL_WARPS - 1) / SEL_WARPS),
+                             dim3(SEL_WARPS * 32), 0, st, a);
+    return e == cudaSuccess ? VELOX_OK : VELOX_ECUDA;
 }
 
 template <typename TIn, int D, int T>
@@ -710,7 +741,7 @@ int route_typed(const TIn* q, const TIn* k, const RouteArgs& r, cudaStream_t st)
         return VELOX_ECUDA;
     SelArgs sa{r.scores, BH * r.m, r.n_past, r.m, r.H, r.P, r.topk - r.m, r.topk,
                r.counts, r.alpha, 1.0f / static_cast<float>(T), r.idx};
-    select_launch(sa, st);
+    if (select_launch(sa, st) != VELOX_OK) return VELOX_ECUDA;
     return cudaGetLastError() == cudaSuccess ? VELOX_OK : VELOX_ECUDA;
 }
 
