@@ -54,7 +54,7 @@ size_t velox_route_topk_workspace_size(int B, int H, int Nq, int Nk, int d, int 
     if (B < 1 || H < 1 || T < 1 || Nq < T || Nq % T || Nk < Nq || Nk % Nq || d < 1) return 0;
     const int m = Nq / T;
     const int n_past = (Nk - Nq) / T;
-    return velox::route_ws_bytes(B, H, m, n_past, d);
+    return velox::route_ws_bytes(B, H, m, n_past, d, T);
 }
 
 int velox_route_topk(const void* q, const void* k, int dtype, int B, int H, int Nq, int Nk, int d,
@@ -95,6 +95,11 @@ int velox_route_topk(const void* q, const void* k, int dtype, int B, int H, int 
     const size_t qbar_bytes = (rows * d * sizeof(float) + 255) & ~static_cast<size_t>(255);
     r.qbar = static_cast<float*>(ws);
     r.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + qbar_bytes);
+    if (velox::route_split_scoring(T, d)) {
+        const size_t scores_bytes =
+            (rows * static_cast<size_t>(r.n_past) * sizeof(float) + 255) & ~static_cast<size_t>(255);
+        r.kbar_ws = reinterpret_cast<float*>(static_cast<char*>(ws) + qbar_bytes + scores_bytes);
+    }
     r.counts_ready = static_cast<cudaEvent_t>(counts_ready);
     return velox::route_launch(q, k, dtype, r, as_stream(stream));
 }

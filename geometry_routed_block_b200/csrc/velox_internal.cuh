@@ -52,8 +52,14 @@ struct RouteArgs {
     cudaEvent_t counts_ready;  // selection waits for it when set
     const float* kbar;         // k-bar cache [B*H][kbar_cap][d], or nullptr: pool K here
     int kbar_cap;              // blocks per (b, h) in the cache
+    float* kbar_ws;            // workspace [B*H][n_past][d] when the scoring is split, else nullptr
 };
-size_t route_ws_bytes(int B, int H, int m, int n_past, int d);
+// Whether routing without a k-bar cache pools every past key block into the
+// workspace first and scores from there (instead of scoring each block as it
+// is pooled): for the block shapes whose scoring per byte of K would hold
+// the stream back.
+bool route_split_scoring(int T, int d);
+size_t route_ws_bytes(int B, int H, int m, int n_past, int d, int T);
 int route_launch(const void* q, const void* k, int dtype, const RouteArgs& r, cudaStream_t st);
 
 int kbar_append_launch(const void* k, int dtype, int BH, int Nk, int Nq, int d, int T, int chunk,
