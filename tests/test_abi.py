@@ -78,6 +78,21 @@ def test_route_topk_rejects(lib):
     assert call(alpha=float("nan")) == -1
 
 
+def test_workspace_holds_pooled_keys_for_64_token_blocks(lib):
+    # 64-token blocks pool every past key block into the workspace before
+    # scoring: beyond q-bar (B*H*m*d) and the scores (B*H*m*n_past) it holds
+    # B*H*n_past*d floats; 128-token blocks score as they pool and need no more
+    B, H, d, Nq = 1, 2, 128, 512
+    for T, Nk in ((64, 5 * 512), (128, 5 * 512)):
+        m, n_past = Nq // T, (Nk - Nq) // T
+        base = 4 * B * H * m * (d + n_past)
+        size = lib.velox_route_topk_workspace_size(B, H, Nq, Nk, d, T)
+        if T == 64:
+            assert size >= base + 4 * B * H * n_past * d
+        else:
+            assert base <= size < base + 4 * B * H * n_past * d
+
+
 def test_workspace_sizes(lib):
     assert lib.velox_route_topk_workspace_size(1, 2, 256, 1280, 64, 64) > 0
     assert lib.velox_route_topk_workspace_size(1, 2, 250, 1280, 64, 64) == 0

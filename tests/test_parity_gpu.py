@@ -557,6 +557,25 @@ def test_t64_routed_attention_pairs_blocks(vx, d):
                              label=f"workload 4, P = 8, T = 64, d = {d} (paired query blocks)")
 
 
+def test_t64_routing_takes_exactly_its_workspace(vx):
+    """64-token routing keeps the pooled past keys in the workspace: the size
+    the library reports is enough (same selection as with room to spare) and
+    256 bytes less is refused."""
+    rng = np.random.default_rng(6464)
+    B, H, T, d, m, P = 1, 2, 64, 128, 6, 5
+    q, k, _ = _random_qkv(rng, B, H, m * T, (P + 1) * m * T, d)
+    q, k = dev(q), dev(k)
+    topk = 13
+    n = vx.lib.velox_route_topk_workspace_size(B, H, m * T, (P + 1) * m * T, d, T)
+    big = torch.empty(n + 4096, dtype=torch.uint8, device="cuda")
+    exact = torch.empty(n, dtype=torch.uint8, device="cuda")
+    want = vx.route_topk(q, k, None, 0.0, topk, T, ws=big)
+    got = vx.route_topk(q, k, None, 0.0, topk, T, ws=exact)
+    assert torch.equal(got, want)
+    with pytest.raises(vx.VeloxError):
+        vx.route_topk(q, k, None, 0.0, topk, T, ws=exact[: n - 256])
+
+
 def test_t64_long_lists_fall_back_to_one_block_per_tile(vx):
     """A routed list longer than two of them fit in the tile's walk (4,096
     blocks): one 64-token block per tile, still exact against the oracle."""
