@@ -378,23 +378,29 @@ class Workload:
         self.cur = 0
 
     def step_ahead(self, ev=None, route=None, next_depth=None, next_cam=None, next_ready=None):
-        """One step with the geometry pipelined one step ahead: routing (its
-        selection waits for the counts built during the previous step), then
+        """One step with the geometry pipelined one step ahead: routing (after
+        the stream waits for the counts built during the previous step), then
         attention; the next step's slices and counts are built on the side stream
         once this step's selection is done, so they run under this step's
         attention instead of competing with the scorer for SMs (the method builds
         slices asynchronously to denoising). next_depth / next_cam: the next
         step's inputs (default: this step's), next_ready: an event they wait for.
-        ev: routing (ev0 -> ev2, including any wait for the counts) and
-        attention (ev2 -> ev3)."""
+        ev: routing (ev0 -> ev2) and attention (ev2 -> ev3)."""
         torch = self.torch
         main = torch.cuda.current_stream()
         if self.cur is None:
             self.prime()
         j = self.cur
+        # the counts were built on the side stream during the previous step's
+        # attention, so they are ready long before this point on the GPU
+        # timeline: the main stream waits for them here (in the step time, not
+        # in the routing interval), and the routing runs without a mid-stream
+        # event wait (which would keep the selection from overlapping the
+        # scorer's tail)
+        main.wait_event(self.geo_ev[j])
         if ev is not None:
             ev[0].record(main)
-        (route or self.route)(ready=self.geo_ev[j], counts=self.counts2[j])
+        (route or self.route)(ready=None, counts=self.counts2[j])
         self.sel_ev[j].record(main)
         if ev is not None:
             ev[2].record(main)
