@@ -126,7 +126,10 @@ VELOX_API int velox_block_overlap(const float* cur_depth, const velox_slice_t* c
                         const velox_slice_t* slices, int B, int P, int F, int Hp, int Wp, int T,
                         int32_t* counts, void* stream);
 
-/* Bytes of scratch velox_route_topk needs for these sizes (0 on bad sizes). */
+/* Bytes of scratch velox_route_topk needs for these sizes (0 on bad sizes):
+ * q-bar (B*H*m*d floats) and the block scores (B*H*m*n_past floats); with
+ * T = 64 also the pooled past keys (B*H*n_past*d floats), which that block
+ * size scores from after pooling them all (see velox_route_topk). */
 VELOX_API size_t velox_route_topk_workspace_size(int B, int H, int Nq, int Nk, int d, int T);
 
 /*
@@ -150,6 +153,9 @@ VELOX_API size_t velox_route_topk_workspace_size(int B, int H, int Nq, int Nk, i
  *   per (b, h, qb): the m current-chunk blocks are always kept and the
  *   topk - m past blocks with the largest s' are added (equal s': the smaller
  *   kb first). topk counts the current blocks.
+ * With T = 128 each key block is scored as it is pooled; with T = 64 (twice the
+ * query blocks per byte of K) every past block is pooled into the workspace
+ * first and scored from there. Both give bit-identical scores.
  * Errors: VELOX_EINVAL for sizes that are not multiples (Nq % T, Nk % Nq),
  * more than 8192 key blocks (Nk/T), topk < m or topk > Nk/T, ws_bytes too
  * small, NULL or misaligned (16 B) pointers; VELOX_EUNSUPPORTED for T not in
