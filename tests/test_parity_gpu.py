@@ -557,6 +557,29 @@ def test_t64_routed_attention_pairs_blocks(vx, d):
                              label=f"workload 4, P = 8, T = 64, d = {d} (paired query blocks)")
 
 
+@pytest.mark.parametrize("T,d", [(64, 128), (64, 64), (128, 64)])
+def test_other_tile_shapes_at_chunk_48(vx, T, d):
+    """The other block sizes and head dims at the headline's 48 past chunks
+    (workload 4's generator with T and d set: the shapes of the bench line's
+    tile_shapes record): routing of two heads against the oracle, and
+    attention on 12 query blocks spread over each head on the oracle's
+    selection (64-token blocks: the two-tile kernel and the split scoring)."""
+    heads = (4, 21)
+    c = synth.make_case(4, P=48, heads=heads, T=T, d=d)
+    s = c.shape
+    sl = vo.slices_build(c.past_depth[0], c.past_poses[0], c.past_intr[0])
+    counts = vo.block_overlap(c.cur_depth, c.cur_cam, sl[None], s.F, s.T)
+    q, k, v = c.q[0], c.k[0], c.v[0]
+    want, s_mod = oracle_route_per_head(q, k, counts, s.alpha, s.topk, s.T)
+    idx = vx.route_topk(dev(q), dev(k), dev(counts), s.alpha, s.topk, s.T)
+    label = f"chunk 48, T = {T}, d = {d}, heads {heads}"
+    ties = compare_selection(idx.cpu().numpy(), want, s_mod, s.m, label=label)
+    assert ties <= tie_bound(2 * s.m)
+    step = max(1, s.m // 12)
+    rows = [(0, i, qb) for i in range(2) for qb in range(0, s.m, step)][:24]
+    attention_rows_vs_oracle(vx, q, k, v, want, s.T, rows, label=label)
+
+
 def test_t64_routing_takes_exactly_its_workspace(vx):
     """64-token routing keeps the pooled past keys in the workspace: the size
     the library reports is enough (same selection as with room to spare) and
