@@ -1285,7 +1285,8 @@ def run_overlap(args):
     point tests per second) and on a stress shape where its float64 ALU work
     dominates: 64 scenes at 256 x 384 (one frame per chunk) against 96 past
     slices, 604 M point tests. Its rate is set against a measured float64 FMA
-    ceiling (velox_fp64_fma_bench)."""
+    ceiling (velox_fp64_fma_bench). Also the multiwarp's candidate splats per
+    second, at the headline size and with 96 past maps of 256 x 384."""
     import torch
     from geometry_routed_block_b200 import velox as vx
     if int(os.environ.get("RANK", "0")) != 0:
@@ -1328,6 +1329,32 @@ def run_overlap(args):
     flops = tests * OVERLAP_FLOPS_PER_TEST + points * OVERLAP_FLOPS_PER_POINT
     achieved = flops / (t_big * 1e-3) / 1e12
     covered = float((counts.sum(-1) > 0).float().mean().item())
+
+    # the multiwarp (recency-priority splat of the past depth maps into the
+    # current view): candidate splats per second at the headline size and with
+    # 96 past maps at the stress grid
+    def multiwarp_rate(past_depth, poses, intr, cur_cam, n_reps):
+        P_, Hp_, Wp_ = past_depth.shape
+        pd = dev(past_depth)
+        cams = dev(np.stack([synth.camera_record(poses[j], intr[j]) for j in range(P_)]))
+        cc = dev(cur_cam)
+        ws = vx.depth_multiwarp_workspace(Hp_, Wp_, device)
+        cur = torch.empty((Hp_, Wp_), dtype=torch.float32, device=device)
+        call = lambda: vx.depth_multiwarp(pd, cams, cc, 0.01, ws=ws, out=cur)
+        for _ in range(3):
+            call()
+        t_ = time_loop(torch, call, n_reps)
+        splats = P_ * Hp_ * Wp_
+        return {"shape": f"{P_} past maps of {Hp_}x{Wp_}", "ms": round(t_, 4), "candidate_splats": splats,
+                "splats_per_s": round(splats / (t_ * 1e-3), 1),
+                "holes_fraction": round(float(torch.isnan(cur).float().mean().item()), 4)}
+
+    geo3 = synth.geometry_only(3)
+    mw_head = multiwarp_rate(geo3.past_depth[0], geo3.past_poses[0], geo3.past_intr[0],
+                             geo3.cur_cam[0], reps)
+    g_mw = synth.stress_geometry(1, 96, Hp, Wp, seed=1011, past_grid=(Hp, Wp))
+    mw_big = multiwarp_rate(g_mw["past_depth"][0], g_mw["past_poses"][0], g_mw["past_intr"][0],
+                            g_mw["cur_cam"][0], 10)
     out = {
         "workload": "slice overlap (step 3 of the method's geometry): headline size and a stress shape",
         "data": "synthetic", "n_gpus": 1,
@@ -1345,6 +1372,9 @@ def run_overlap(args):
                      "unit": "TFLOP/s", "frac": round(achieved / fp64_peak, 4),
                      "peak_kind": "measured float64 FMA rate (velox_fp64_fma_bench, FMA = 2 FLOP)",
                      "traffic": None},
+        "multiwarp": {"headline": mw_head, "stress": mw_big,
+                      "note": "every valid past pixel is a candidate: back-projection, projection and "
+                              "64-bit atomic minima on the target pixel (float64 geometry)"},
     }
     print(json.dumps(out), flush=True)
 
