@@ -79,6 +79,13 @@ struct PRBars {
     __device__ uint32_t mma_drain() const { return base + 8 * 13; }
 };
 
+// Pairs 0 and 4 of every 8 go to the FMA pipe (Cody-Waite cubic), the rest to
+// the ex2 unit. This kernel's MMA chain has room to spare, so its softmax sets
+// the pace, and taking a quarter of the exponentials off the ex2 unit shortens
+// it: 12 alternating rounds, chunk 48 / P = 8, routed 995 -> 1,061 / 957 -> 999
+// and dense 1,101 -> 1,109 / 1,075 -> 1,130 TFLOP/s.
+constexpr unsigned PR_EMU_MASK = 0x11;
+
 // exponentials of 64 scores (one half row) in place, sums into sum2
 __device__ __forceinline__ void pr_exp_half(float* s, float sl2, float m, float2* sum2) {
     const float2 sc2 = make_float2(sl2, sl2);
@@ -86,8 +93,12 @@ __device__ __forceinline__ void pr_exp_half(float* s, float sl2, float m, float2
 #pragma unroll
     for (int i = 0; i < 64; i += 2) {
         float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), sc2, ng2);
-        x.x = ex2_approx(x.x);
-        x.y = ex2_approx(x.y);
+        if ((PR_EMU_MASK >> ((i >> 1) & 7)) & 1) {
+            x = exp2_poly2(x);
+        } else {
+            x.x = ex2_approx(x.x);
+            x.y = ex2_approx(x.y);
+        }
         s[i] = x.x;
         s[i + 1] = x.y;
         sum2[(i >> 1) & 3] = __fadd2_rn(sum2[(i >> 1) & 3], x);

@@ -101,7 +101,10 @@ def test_walk_dense_attention_rows(vx, walk):
     rows = [(0, h, qb) for h in (0, 5, 11) for qb in (0, 17, 35)]
     ref = vo.sparse_attention(walk.q[0], walk.k[0], walk.v[0], None, s.T, rows=rows)
     o, lse = vx.sparse_attn_fwd(q, k, v, None, s.T)
-    # top-k = every block, listed explicitly, is the same computation
+    # top-k = every block, listed explicitly, is the same computation (on the
+    # two-block kernel; the dense walk runs on the CTA-pair kernel, which takes
+    # a quarter of its exponentials on the FMA pipe, so the two agree to a few
+    # bf16 units in the last place rather than bit for bit)
     all_idx = torch.arange(s.nKB, dtype=torch.int32, device="cuda").expand(s.B, s.H, s.m, s.nKB)
     o2, _ = vx.sparse_attn_fwd(q, k, v, all_idx.contiguous(), s.T)
     for (b, h, qb), (o_ref, lse_ref) in ref.items():
@@ -109,7 +112,7 @@ def test_walk_dense_attention_rows(vx, walk):
         compare_attention(o[b, h, sl], o_ref, f"dense row {(b, h, qb)}")
         compare_attention(o2[b, h, sl], o_ref, f"all-listed row {(b, h, qb)}")
         assert np.abs(lse[b, h, sl].cpu().numpy() - lse_ref).max() < 1e-3
-    assert torch.equal(o, o2)
+    assert float((o.float() - o2.float()).abs().max()) <= 4e-3
 
 
 def test_walk_routing_alpha0_and_geometry(vx, walk):
