@@ -8,8 +8,8 @@ with the KV cache resident in HBM: frustum slices of every past chunk, slice
 overlap counts, geometry-modulated top-k routing (pooling + scores + select)
 and block-sparse attention over the routed blocks. The slices and counts are
 built on a side stream one step ahead: chunk n+1's are built while chunk n's
-attention runs (the selection of a step waits only for its own counts, built
-during the step before), as the method builds its slices asynchronously to
+attention runs (a step's routing waits only for its own counts, built during
+the step before), as the method builds its slices asynchronously to
 denoising; the timed steps therefore hold one extra geometry pass (the next
 chunk's). `value` is the whole-job throughput in TFLOP/s of attention work on
 the kept blocks
