@@ -120,7 +120,11 @@ def routing_bytes(s: synth.Shape) -> float:
 # ----------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi queries (read only) every 50 ms while it is open; begin() and
+    end() mark the timed region on the host clock, and summary() keeps the
+    samples taken inside it (all of them, flagged, if the region was shorter
+    than the sampling interval)."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -128,6 +132,13 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
+
+    def begin(self):
+        self.t0 = time.time()
+
+    def end(self):
+        self.t1 = time.time()
 
     def __enter__(self):
         try:
@@ -136,7 +147,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
@@ -154,23 +165,33 @@ class ClockSampler:
     def summary(self):
         if self.proc is None or not self.path or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sm, smax, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        import datetime
+        rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
+            if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[0]))
-                smax = float(parts[1])
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[4:8]):
+        os.unlink(self.path)
+        inside = [r for r in rows if self.t0 is not None and self.t1 is not None
+                  and self.t0 <= r[0] <= self.t1]
+        use = inside if inside else rows
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = set()
+        for r in use:
+            for n, v in zip(names, r[3]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        sm = [r[1] for r in use]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": use[-1][2] if use else None, "samples": len(sm),
+                "window": "timed region" if inside else "whole sampler run (no sample inside "
+                                                        "the timed region)",
+                "reasons": sorted(reasons)}
 
 
 # ----------------------------------------------------------------------------
@@ -577,12 +598,14 @@ def run_gpu(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
+        clk.begin()
         t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t_start.record()
         for i in range(args.steps):
             w.step_ahead(evs[i])
         t_end.record()
         torch.cuda.synchronize()
+        clk.end()
         if world > 1:
             dist.barrier()
     clocks = clk.summary()
@@ -956,7 +979,9 @@ def pipeline_measure(torch, vx, device, layers: int, steps: int, warmup: int, se
     steps = max(1, steps)
     # the timed region: K whole steps with the geometry in flight on the side stream
     with ClockSampler(device.index or 0) as clk:
+        clk.begin()
         t_async = time_loop(torch, step_async, steps)
+        clk.end()
     clocks = clk.summary()
     # exposure, per step, from events: when the geometry is done vs when layer 0's
     # routing (whose selection waited for it) is done; plus the same steps run
